@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE dispatch/combine hot path (layout -> dispatch -> combine)
+on the DeepSeek-V3-shaped low-latency decode workload: 8 logical ranks x 128
+tokens (B = 1024), d = 7168, E = 256, top-8, int8 dynamic quantization.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode] [--flush-mb 512] [--no-cpu-baseline]
+
+One step = one pass of the whole path over one batch: ep_layout, ep_dispatch,
+ep_combine through the C ABI.  The expert output buffer that combine reads is
+resident (the identity expert: the dequantized receive rows), since the expert
+computation is not part of dispatch/combine.  L2 is flushed (a 512 MB memset)
+between timed steps, outside the per-step events.
+
+Prints one JSON line (rank 0).  value = algorithmic HBM bytes of the three
+kernels / step time, whole job (all ranks), in GB/s.
+--impl reference times the CPU oracle (the reference arm for this path) on the
+host cores, one bounded sample of the workload per step.
+With N > 1 (torchrun), every rank runs an independent replica (the EP ranks are
+logical partitions of one GPU; nothing is exchanged between GPUs).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine HBM GB/s and tokens/s at d=7168,E=256,k=8; % of B200 HBM peak"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+PROFILES = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = {
+    "layout": "combine_ep_layout_12_b200/csrc/ep_layout.cu",
+    "dispatch": "combine_ep_layout_12_b200/csrc/ep_dispatch.cu",
+    "combine": "combine_ep_layout_12_b200/csrc/ep_combine.cu",
+}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="decode")
+    p.add_argument("--flush-mb", type=int, default=512)
+    p.add_argument("--e2e-steps", type=int, default=None, help="steps of the end-to-end loop (default min(K, 200))")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
+    return p.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def aggregate(dist, seconds, units, device=None):
+    """Whole-job numbers over ranks: time = max over ranks, units = sum over ranks."""
+    if dist is None:
+        return seconds, units
+    import torch
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_power_brake": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, index, period=0.01):
+        self.samples = []
+        self.period = period
+        self.ok = False
+        self.window = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as exc:  # no NVML: report that instead of numbers
+            self.error = repr(exc)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.th.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "error", "")}
+        t0, t1 = self.window if self.window else (-1e30, 1e30)
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        used = inside
+        note = None
+        if len(inside) < 3:  # short timed region: widen to the neighbouring samples
+            used = sorted(self.samples, key=lambda s: abs(s[0] - 0.5 * (t0 + t1)))[:5]
+            note = "timed region shorter than the sampling period; nearest samples used"
+        mhz = [s[1] for s in used]
+        reasons = set()
+        for s in used:
+            for name, attr in self.REASONS.items():
+                bit = getattr(self.nv, attr, 0)
+                if bit and (s[2] & bit):
+                    reasons.add(name)
+        out = {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+               "reasons": sorted(reasons), "samples": len(used)}
+        if note:
+            out["note"] = note
+        return out
+
+
+# ----------------------------------------------------------------------------- helpers
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(name):
+    with open(os.path.join(ROOT, KERNEL_SOURCES[name]), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(PROFILES, "traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        rec = j[workload][kernel]
+        if rec.get("source_sha") != source_hash(kernel):
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def oracle_step_sample(w, inp, n_tokens):
+    """One oracle pass (layout, quantize, scatter, combine) over the first
+    n_tokens tokens (a whole number of ranks' worth if possible).  Returns
+    (seconds, algorithmic bytes of that sample)."""
+    import oracle
+    from combine_ep_layout_12_b200 import metrics
+    B = n_tokens
+    P = max(1, min(w.P, B // max(1, w.T)))
+    if B % P:
+        P = 1
+    M = max(w.M, B // P)
+    cfg = oracle.make_cfg(B, w.d, w.k, P, M, w.E, w.n_zero, w.n_copy, w.n_const, w.quant_mode)
+    idx = np.ascontiguousarray(inp["topk_idx"][:B])
+    x = np.ascontiguousarray(inp["x"][:B])
+    wts = np.ascontiguousarray(inp["topk_weights"][:B])
+    t0 = time.perf_counter()
+    lay = oracle.layout(cfg, idx)
+    q, ts = oracle.quantize(cfg, x, inp["smooth"])
+    # scatter into a compact receive buffer (one row per routed pick, same bytes)
+    dp = lay["dst_pos"]
+    compact = np.full(dp.shape, -1, np.int32)
+    routed = dp >= 0
+    n_r = int(routed.sum())
+    compact[routed] = np.arange(n_r, dtype=np.int32)
+    rx, rsc = oracle.dispatch(cfg, q, ts, compact, max(n_r, 1))
+    t1 = time.perf_counter()
+    # stand-in expert outputs (bf16 bit patterns) for combine; not part of the
+    # method and not timed
+    if w.quant_mode == 2:
+        eo = np.zeros((max(n_r, 1), w.d), np.uint16)
+        if n_r:
+            f = rx[:n_r].astype(np.float32) * rsc[:n_r, None]
+            eo[:n_r] = (f.view(np.uint32) >> 16).astype(np.uint16)
+    else:
+        eo = rx
+    t2 = time.perf_counter()
+    y = oracle.combine(cfg, eo, idx, wts, compact, x, inp["a1"], inp["a2"], inp["v"])
+    t3 = time.perf_counter()
+    del y
+    nr, bsp = metrics.routing_counts(w.with_(B=B), idx, n_r)
+    by = metrics.kernel_bytes(w.with_(B=B, P=P, M=M), nr, bsp, smooth=inp["smooth"] is not None)
+    return (t1 - t0) + (t3 - t2), sum(by.values())
+
+
+def cpu_baseline(w, inp, target_s):
+    n_tok = min(w.B, max(w.T, 1))
+    secs, nbytes, reps = 0.0, 0, 0
+    while secs < target_s or reps < 1:
+        s, b = oracle_step_sample(w, inp, n_tok)
+        secs += s
+        nbytes += b
+        reps += 1
+        if reps >= 1000:
+            break
+    return {"value": nbytes / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": "%d oracle passes over the first %d tokens (one logical rank) of the %s "
+                      "workload, single-threaded C, %.1f s" % (reps, n_tok, w.name, secs)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    from combine_ep_layout_12_b200 import workloads as wl
+    w = wl.get(args.workload)
+    inp = wl.generate(w)
+    n_tok = min(w.B, max(w.T, 1))
+    for _ in range(args.warmup):
+        oracle_step_sample(w, inp, n_tok)
+    secs, nbytes = 0.0, 0
+    for _ in range(args.steps):
+        s, b = oracle_step_sample(w, inp, n_tok)
+        secs += s
+        nbytes += b
+    value = nbytes / secs / 1e9
+    sample = "%d oracle passes over the first %d tokens (one logical rank) of the %s workload, " \
+             "single-threaded C" % (args.steps, n_tok, w.name)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": config_dict(w, args),
+        "tokens_per_s": n_tok * args.steps / secs,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, args):
+    return {"workload": w.name, "B": w.B, "d": w.d, "E": w.E, "k": w.k, "P": w.P, "M": w.M,
+            "n_zero": w.n_zero, "n_copy": w.n_copy, "n_const": w.n_const,
+            "quant_mode": w.quant_mode, "payload": "int8" if w.quant_mode == 2 else "bf16",
+            "routing": w.routing, "layout": "low-latency [E, P*M, d]",
+            "l2": ("flushed between steps (%d MB memset, outside the step events)" % args.flush_mb)
+            if args.flush_mb else "not flushed",
+            "parallelism": "replicas (logical EP ranks inside each GPU)"}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+
+def run_ours(args):
+    import torch
+    from combine_ep_layout_12_b200 import build as ep_build
+    from combine_ep_layout_12_b200 import metrics, runner
+    from combine_ep_layout_12_b200 import workloads as wl
+
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    ep_build.build()
+
+    w = wl.get(args.workload)
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, device)
+    stream = torch.cuda.Stream(device)
+    pipe = runner.Pipeline(w, device)
+
+    # identity expert: expert_out rows = dequantized receive rows (setup, not timed)
+    with torch.cuda.stream(stream):
+        pipe.layout(dev_inp, stream)
+        pipe.dispatch(dev_inp, stream)
+    stream.synchronize()
+    assert pipe.buf.check() == 0, "device error bits set"
+    dp = pipe.buf.dst_pos
+    rows = dp[dp >= 0].long()
+    if w.quant_mode == 2:
+        deq = pipe.buf.recv_x[rows].float() * pipe.buf.recv_scale[rows].unsqueeze(1)
+        pipe.expert_out[rows] = deq.to(torch.bfloat16)
+    n_routed = int(rows.numel())
+    n_routed_chk, b_sp = metrics.routing_counts(w, inp["topk_idx"], n_routed)
+    kbytes = metrics.kernel_bytes(w, n_routed, b_sp, smooth=inp["smooth"] is not None)
+    step_bytes = sum(kbytes.values())
+
+    flush = torch.empty(max(args.flush_mb, 1) << 20, dtype=torch.uint8, device=device) if args.flush_mb else None
+
+    def one_step(ev=None):
+        if flush is not None:
+            flush.zero_()
+        if ev is not None:
+            ev[0].record(stream)
+        pipe.layout(dev_inp, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        pipe.dispatch(dev_inp, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        pipe.combine(dev_inp, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one_step()
+    stream.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(device.index if device.index is not None else 0)
+    clocks.start()
+    time.sleep(0.05)
+    barrier(dist, device)
+    torch.cuda.synchronize(device)
+    t_wall0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            one_step(evs[i])
+    torch.cuda.synchronize(device)
+    t_wall1 = time.perf_counter()
+    barrier(dist, device)
+    clocks.mark(t_wall0, t_wall1)
+    time.sleep(0.03)
+    clocks.stop()
+    assert pipe.buf.check(stream) == 0, "device error bits set during the timed steps"
+
+    per = {"layout": [], "dispatch": [], "combine": []}
+    step_ms = []
+    for ev in evs:
+        per["layout"].append(ev[0].elapsed_time(ev[1]))
+        per["dispatch"].append(ev[1].elapsed_time(ev[2]))
+        per["combine"].append(ev[2].elapsed_time(ev[3]))
+        step_ms.append(ev[0].elapsed_time(ev[3]))
+    local_s = sum(step_ms) / 1e3
+    job_s, job_bytes = aggregate(dist, local_s, float(step_bytes * K), device)
+    _, job_tokens = aggregate(dist, local_s, float(w.B * K), device)
+    value = job_bytes / job_s / 1e9
+
+    # per-kernel roofline (this rank)
+    peak, peak_kind = measured_peak()
+    kernels = {}
+    for name in ("layout", "dispatch", "combine"):
+        ms = statistics.mean(per[name])
+        ach = kbytes[name] / (ms * 1e-3) / 1e9
+        kernels[name] = {"us_mean": 1e3 * ms, "us_median": 1e3 * statistics.median(per[name]),
+                         "bytes": kbytes[name], "achieved_gbs": ach,
+                         "frac_of_measured": ach / peak, "frac_of_8tbs": ach / SPEC_HBM_GBS,
+                         "share": sum(per[name]) / sum(step_ms)}
+    dom = max(("dispatch", "combine", "layout"), key=lambda n: kernels[n]["share"])
+    traffic = recorded_traffic(w.name, dom)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["achieved_gbs"], "peak": peak,
+                "unit": "GB/s", "frac": kernels[dom]["achieved_gbs"] / peak, "traffic": traffic,
+                "peak_source": "%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peak_kind
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "frac_of_8tbs_spec": kernels[dom]["achieved_gbs"] / SPEC_HBM_GBS,
+                "algorithmic_bytes": kbytes[dom]}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Ke = args.e2e_steps if args.e2e_steps is not None else min(K, 200)
+        host = runner.to_device(inp, device, pin=True)
+        y_host = torch.empty((w.B, w.d), dtype=torch.bfloat16).pin_memory()
+        names = [n for n in ("x", "topk_idx", "topk_weights") if dev_inp.get(n) is not None]
+        h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+        d2h = y_host.numel() * y_host.element_size()
+        e0 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+        e1 = [torch.cuda.Event(enable_timing=True) for _ in range(Ke)]
+        barrier(dist, device)
+        torch.cuda.synchronize(device)
+        with torch.cuda.stream(stream):
+            for i in range(Ke):
+                if flush is not None:
+                    flush.zero_()
+                e0[i].record(stream)
+                for n in names:
+                    dev_inp[n].copy_(host[n], non_blocking=True)
+                pipe.step(dev_inp, stream)
+                y_host.copy_(pipe.y, non_blocking=True)
+                e1[i].record(stream)
+        torch.cuda.synchronize(device)
+        barrier(dist, device)
+        loc = sum(a.elapsed_time(b) for a, b in zip(e0, e1)) / 1e3
+        js, jb = aggregate(dist, loc, float(step_bytes * Ke), device)
+        e2e = {"value": jb / js / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": Ke, "ms_per_step": 1e3 * js / Ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp, args.cpu_seconds)
+
+    if dist is not None:
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": 1e3 * job_s / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_dict(w, args),
+        "tokens_per_s": job_tokens / job_s,
+        "bytes_per_step": step_bytes,
+        "kernels": kernels,
+        "comm_gbs_dispatch": n_routed * w.d * (1 if w.quant_mode == 2 else 2)
+        / (statistics.mean(per["dispatch"]) * 1e-3) / 1e9,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clocks.summary(),
+        "gpu_launches": 3 * K,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,132 @@
-"""B200-native MoE expert-parallel dispatch and combine (logical EP ranks on one GPU)."""
+"""B200-native MoE expert-parallel token dispatch and combine, with the EP ranks
+as logical partitions of one GPU's memory.
+
+The compute path is libep.so (CUDA kernels for sm_100a behind the C ABI of
+include/ep.h).  `_binding` holds the one-to-one ctypes functions; `EPBuffer`
+below is a convenience wrapper that allocates the caller-owned arrays as torch
+tensors and passes their addresses through.  torch supplies device memory and
+streams only.  There is no CPU or torch fallback: every call fails loudly if
+libep.so is missing.
+"""
+import torch
+
+from . import _binding as abi
+from ._binding import (EPError, ep_buffer_check, ep_buffer_create, ep_buffer_destroy,
+                       ep_buffer_size, ep_combine, ep_dispatch, ep_layout, ep_status_str,
+                       make_config)
+
+__all__ = ["EPBuffer", "EPError", "abi", "ep_buffer_check", "ep_buffer_create",
+           "ep_buffer_destroy", "ep_buffer_size", "ep_combine", "ep_dispatch", "ep_layout",
+           "ep_status_str", "make_config"]
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _need(t, name, dtype, shape, device):
+    if t is None:
+        raise ValueError("%s is required" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.device != device:
+        raise ValueError("%s must be on %s, got %s" % (name, device, t.device))
+    return t
+
+
+class EPBuffer:
+    """Caller-owned arrays of one dispatch/combine problem plus the libep handle.
+
+    cfg: an ep_config (see make_config) or any object with the config fields
+    (B, d, k, P, M, E, n_zero, n_copy, n_const, quant_mode[, smooth_rows]).
+    Views: expert_count [E_tot], expert_offset [E_tot+1], recv_count [E, P],
+    dst_pos [B, k], recv_src [E*P*M], recv_x [E*P*M, d] (int8 or bf16),
+    recv_scale [E*P*M], token_scale [B].
+    """
+
+    def __init__(self, cfg, device=None):
+        if not isinstance(cfg, abi.ep_config):
+            cfg = make_config(cfg.B, cfg.d, cfg.k, cfg.P, cfg.M, cfg.E, cfg.n_zero, cfg.n_copy,
+                              cfg.n_const, cfg.quant_mode, getattr(cfg, "smooth_rows", 1), 0)
+        self.cfg = cfg
+        dev = torch.device("cuda" if device is None else device)
+        if dev.type != "cuda":
+            raise ValueError("EPBuffer lives on a CUDA device, got %s" % dev)
+        self.device = dev if dev.index is not None else torch.device("cuda", torch.cuda.current_device())
+        sizes = ep_buffer_size(cfg)
+        self.sizes = {n: int(getattr(sizes, n)) for n in abi.BUFFER_FIELDS}
+        c = cfg
+        self.E_tot = c.E + c.n_zero + c.n_copy + c.n_const
+        self.rows = c.E * c.P * c.M
+        dev = self.device
+        self.expert_count = torch.empty(self.E_tot, dtype=torch.int32, device=dev)
+        self.expert_offset = torch.empty(self.E_tot + 1, dtype=torch.int32, device=dev)
+        self.recv_count = torch.empty((c.E, c.P), dtype=torch.int32, device=dev)
+        self.dst_pos = torch.empty((c.B, c.k), dtype=torch.int32, device=dev)
+        self.recv_src = torch.empty(self.rows, dtype=torch.int32, device=dev)
+        xdt = torch.int8 if c.quant_mode == 2 else torch.bfloat16
+        self.recv_x = torch.empty((self.rows, c.d), dtype=xdt, device=dev)
+        q = c.quant_mode == 2
+        self.recv_scale = torch.empty(self.rows, dtype=torch.float32, device=dev) if q else None
+        self.token_scale = torch.empty(c.B, dtype=torch.float32, device=dev) if q else None
+        self.workspace = torch.empty(self.sizes["workspace"], dtype=torch.uint8, device=dev)
+        ptrs = abi.ep_buffer_ptrs(*[_ptr(getattr(self, n)) for n in abi.BUFFER_FIELDS])
+        with torch.cuda.device(dev):
+            self.handle = ep_buffer_create(cfg, ptrs)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            ep_buffer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- hot path ---------------------------------------------------------------
+    def layout(self, topk_idx, stream=None):
+        c = self.cfg
+        _need(topk_idx, "topk_idx", torch.int32, (c.B, c.k), self.device)
+        ep_layout(self.handle, _ptr(topk_idx), _stream(stream))
+
+    def dispatch(self, x, smooth_scale=None, stream=None):
+        c = self.cfg
+        _need(x, "x", torch.bfloat16, (c.B, c.d), self.device)
+        if smooth_scale is not None:
+            _need(smooth_scale, "smooth_scale", torch.float32, (c.d,), self.device)
+        ep_dispatch(self.handle, _ptr(x), _ptr(smooth_scale), _stream(stream))
+
+    def combine(self, expert_out, topk_idx, topk_weights, ori_x=None, a1=None, a2=None, v=None,
+                y=None, stream=None):
+        c = self.cfg
+        _need(expert_out, "expert_out", torch.bfloat16, (self.rows, c.d), self.device)
+        _need(topk_idx, "topk_idx", torch.int32, (c.B, c.k), self.device)
+        _need(topk_weights, "topk_weights", torch.float32, (c.B, c.k), self.device)
+        if c.n_copy + c.n_const > 0:
+            _need(ori_x, "ori_x", torch.bfloat16, (c.B, c.d), self.device)
+        if c.n_const > 0:
+            for n, t in (("a1", a1), ("a2", a2), ("v", v)):
+                _need(t, n, torch.bfloat16, (c.n_const, c.d), self.device)
+        if y is None:
+            y = torch.empty((c.B, c.d), dtype=torch.bfloat16, device=self.device)
+        else:
+            _need(y, "y", torch.bfloat16, (c.B, c.d), self.device)
+        ep_combine(self.handle, _ptr(expert_out), _ptr(topk_idx), _ptr(topk_weights), _ptr(ori_x),
+                   _ptr(a1), _ptr(a2), _ptr(v), _ptr(y), _stream(stream))
+        return y
+
+    def check(self, stream=None):
+        """Synchronize and return (and clear) the device error bits."""
+        return ep_buffer_check(self.handle, _stream(stream))

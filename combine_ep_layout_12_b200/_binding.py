@@ -1,0 +1,124 @@
+"""ctypes binding of libep.so: the C ABI of include/ep.h, one Python function per
+entry point with the same name.  Argument marshalling only; every step of the
+path runs in the library's CUDA kernels.  Pointers are passed as Python ints
+(device addresses); streams as cudaStream_t handles (ints, 0 = default stream).
+"""
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libep.so")
+
+EP_OK = 0
+EP_ERR_INVALID_ARG = -1
+EP_ERR_UNSUPPORTED = -2
+EP_ERR_CAPACITY = -3
+EP_ERR_CUDA = -4
+
+ERRBIT_BAD_ID = 0x1
+ERRBIT_DUP_ID = 0x2
+ERRBIT_ROW_RANGE = 0x4
+
+_CONFIG_FIELDS = ("B", "d", "k", "P", "M", "E", "n_zero", "n_copy", "n_const", "quant_mode",
+                  "smooth_rows", "layout")
+BUFFER_FIELDS = ("expert_count", "expert_offset", "recv_count", "dst_pos", "recv_src", "recv_x",
+                 "recv_scale", "token_scale", "workspace")
+
+
+class ep_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in _CONFIG_FIELDS]
+
+
+class ep_buffer_sizes(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in BUFFER_FIELDS]
+
+
+class ep_buffer_ptrs(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_FIELDS]
+
+
+class EPError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)" % (where, ep_status_str(status), status))
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libep.so.  Raises if the library has not been built: there is no
+    fallback implementation."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libep.so is missing at %s; build it with "
+                           "`python -m combine_ep_layout_12_b200.build`" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    L.ep_buffer_size.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_buffer_sizes)]
+    L.ep_buffer_create.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_buffer_ptrs),
+                                   ctypes.POINTER(vp)]
+    L.ep_buffer_destroy.argtypes = [vp]
+    L.ep_layout.argtypes = [vp, vp, vp]
+    L.ep_dispatch.argtypes = [vp, vp, vp, vp]
+    L.ep_combine.argtypes = [vp] * 10
+    L.ep_buffer_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    for f in (L.ep_buffer_size, L.ep_buffer_create, L.ep_buffer_destroy, L.ep_layout,
+              L.ep_dispatch, L.ep_combine, L.ep_buffer_check):
+        f.restype = i
+    L.ep_status_str.argtypes = [i]
+    L.ep_status_str.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def make_config(B, d, k, P, M, E, n_zero=0, n_copy=0, n_const=0, quant_mode=0, smooth_rows=0,
+                layout=0):
+    return ep_config(B, d, k, P, M, E, n_zero, n_copy, n_const, quant_mode, smooth_rows, layout)
+
+
+def _check(status, where):
+    if status != EP_OK:
+        raise EPError(status, where)
+
+
+def ep_status_str(status):
+    return lib().ep_status_str(int(status)).decode()
+
+
+def ep_buffer_size(cfg):
+    out = ep_buffer_sizes()
+    _check(lib().ep_buffer_size(ctypes.byref(cfg), ctypes.byref(out)), "ep_buffer_size")
+    return out
+
+
+def ep_buffer_create(cfg, ptrs):
+    h = ctypes.c_void_p()
+    _check(lib().ep_buffer_create(ctypes.byref(cfg), ctypes.byref(ptrs), ctypes.byref(h)),
+           "ep_buffer_create")
+    return h
+
+
+def ep_buffer_destroy(handle):
+    _check(lib().ep_buffer_destroy(handle), "ep_buffer_destroy")
+
+
+def ep_layout(handle, topk_idx, stream=0):
+    _check(lib().ep_layout(handle, topk_idx, stream), "ep_layout")
+
+
+def ep_dispatch(handle, x, smooth_scale=None, stream=0):
+    _check(lib().ep_dispatch(handle, x, smooth_scale, stream), "ep_dispatch")
+
+
+def ep_combine(handle, expert_out, topk_idx, topk_weights, ori_x, a1, a2, v, y, stream=0):
+    _check(lib().ep_combine(handle, expert_out, topk_idx, topk_weights, ori_x, a1, a2, v, y,
+                            stream), "ep_combine")
+
+
+def ep_buffer_check(handle, stream=0):
+    bits = ctypes.c_uint32()
+    _check(lib().ep_buffer_check(handle, stream, ctypes.byref(bits)), "ep_buffer_check")
+    return int(bits.value)

@@ -1,0 +1,180 @@
+// Combine kernel: the weighted gather-reduce of expert outputs back to tokens,
+// with the zero, copy and constant special experts (Ascend CANN
+// "low_latency_dispatch", Formula, special expert scenario: Moe(ori_x) = 0,
+// Moe(ori_x) = ori_x, Moe(ori_x) = alpha1 * ori_x + alpha2 * v; low_latency_combine
+// takes the dispatch outputs, topk_weights and ori_x).
+//
+//   y[t] = bf16_rn( acc ),  acc = 0;  for j = 0..k-1 in order:
+//          acc = fma(w[t][j], e(t,j), acc)   (fp32, one rounding per pick)
+//   e = fp32(expert_out[dst_pos[t][j]])          routed pick
+//       fp32(ori_x[t])                            copy expert
+//       a1[c]*ori_x[t] + a2[c]*v[c]  (fp32 ops)   constant expert c
+//   -1, zero experts, dropped picks: no term.
+//
+// Design.  A CTA covers NT consecutive 16-byte column vectors (8 bf16) of one
+// token.  The token's k picks are classified once into shared memory, then each
+// thread issues all k 16-byte loads of its column before accumulating, so a
+// thread keeps k loads in flight; the k-order fused multiply-adds match the
+// definition exactly.
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+enum : int { kSkip = 0, kRouted = 1, kCopy = 2, kConst = 3 };
+
+struct CombineArgs {
+    const uint16_t* expert_out;  // [rows][d]
+    const int32_t* topk_idx;     // [B][k]
+    const float* topk_weights;   // [B][k]
+    const int32_t* dst_pos;      // [B][k]
+    const uint16_t* ori_x;       // [B][d]
+    const uint16_t* a1;          // [K][d]
+    const uint16_t* a2;
+    const uint16_t* v;
+    uint16_t* y;                 // [B][d]
+    unsigned* err;
+    long long rows;
+    int d, k, E, Z, C, K;
+    int chunks;                  // CTAs per token
+};
+
+__device__ __forceinline__ void unpack8(const uint4& r, float* f) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = bf16lo(w[i]);
+        f[2 * i + 1] = bf16hi(w[i]);
+    }
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
+    __shared__ int s_kind[KMAX];
+    __shared__ long long s_src[KMAX];  // receive row (routed) or const index
+    __shared__ float s_w[KMAX];
+
+    const int t = blockIdx.x / a.chunks;
+    const int chunk = blockIdx.x - t * a.chunks;
+    const int nvec = a.d >> 3;
+    const int vcol = chunk * blockDim.x + threadIdx.x;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    unsigned bad = 0;
+    if (threadIdx.x < a.k) {
+        const size_t i = (size_t)t * a.k + threadIdx.x;
+        const int g = a.topk_idx[i];
+        const int dp = a.dst_pos[i];
+        int kind = kSkip;
+        long long src = 0;
+        if (g >= 0 && g < a.E) {
+            if (dp >= 0 && (long long)dp < a.rows) {
+                kind = kRouted;
+                src = dp;
+            } else if (dp != -1) {
+                bad = EP_ERRBIT_ROW_RANGE;
+            }
+        } else if (g >= a.E + a.Z && g < a.E + a.Z + a.C) {
+            kind = kCopy;
+        } else if (g >= a.E + a.Z + a.C && g < a.E + a.Z + a.C + a.K) {
+            kind = kConst;
+            src = g - (a.E + a.Z + a.C);
+        }
+        s_kind[threadIdx.x] = kind;
+        s_src[threadIdx.x] = src;
+        s_w[threadIdx.x] = a.topk_weights[i];
+    }
+    if (threadIdx.x < 32) report_err(a.err, bad);
+    __syncthreads();
+    if (vcol >= nvec) return;
+
+    const size_t col = (size_t)vcol * 8;
+    uint4 raw[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        raw[j] = make_uint4(0, 0, 0, 0);
+        if (j < a.k) {
+            const int kind = s_kind[j];
+            if (kind == kRouted)
+                raw[j] = ld_stream_v4(a.expert_out + (size_t)s_src[j] * a.d + col);
+            else if (kind != kSkip)
+                raw[j] = ld_stream_v4(a.ori_x + (size_t)t * a.d + col);
+        }
+    }
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        if (j >= a.k) continue;
+        const int kind = s_kind[j];
+        if (kind == kSkip) continue;
+        float e[8];
+        unpack8(raw[j], e);
+        if (kind == kConst) {
+            const size_t off = (size_t)s_src[j] * a.d + col;
+            float f1[8], f2[8], fv[8];
+            unpack8(ld_stream_v4(a.a1 + off), f1);
+            unpack8(ld_stream_v4(a.a2 + off), f2);
+            unpack8(ld_stream_v4(a.v + off), fv);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) e[i] = __fadd_rn(__fmul_rn(f1[i], e[i]), __fmul_rn(f2[i], fv[i]));
+        }
+        const float w = s_w[j];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(w, e[i], acc[i]);
+    }
+    uint4 out;
+    out.x = pack_bf16x2(acc[0], acc[1]);
+    out.y = pack_bf16x2(acc[2], acc[3]);
+    out.z = pack_bf16x2(acc[4], acc[5]);
+    out.w = pack_bf16x2(acc[6], acc[7]);
+    st_v4(a.y + (size_t)t * a.d + col, out);
+}
+
+}  // namespace
+
+int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
+                   const int32_t* topk_idx, const float* topk_weights, const uint16_t* ori_x,
+                   const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
+                   cudaStream_t stream) {
+    if (s.B == 0) return EP_OK;
+    CombineArgs a;
+    a.expert_out = expert_out;
+    a.topk_idx = topk_idx;
+    a.topk_weights = topk_weights;
+    a.dst_pos = p.dst_pos;
+    a.ori_x = ori_x;
+    a.a1 = a1;
+    a.a2 = a2;
+    a.v = v;
+    a.y = y;
+    a.err = &reinterpret_cast<WsHeader*>(p.workspace)->err;
+    a.rows = s.rows;
+    a.d = s.d;
+    a.k = s.k;
+    a.E = s.E;
+    a.Z = s.Z;
+    a.C = s.C;
+    a.K = s.K;
+    const int nvec = s.d / 8;
+    int NT = nvec < 128 ? ((nvec + 31) / 32) * 32 : 128;
+    a.chunks = (nvec + NT - 1) / NT;
+    const long long nblocks = (long long)s.B * a.chunks;
+    if (nblocks > 0x7fffffffLL) return EP_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)nblocks);
+    cudaError_t e;
+    if (s.k <= 2)
+        e = launch_pdl(combine_kernel<2>, grid, dim3(NT), 0, stream, a);
+    else if (s.k <= 4)
+        e = launch_pdl(combine_kernel<4>, grid, dim3(NT), 0, stream, a);
+    else if (s.k <= 8)
+        e = launch_pdl(combine_kernel<8>, grid, dim3(NT), 0, stream, a);
+    else
+        e = launch_pdl(combine_kernel<16>, grid, dim3(NT), 0, stream, a);
+    return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+}  // namespace ep

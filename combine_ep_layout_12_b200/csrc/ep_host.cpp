@@ -1,0 +1,167 @@
+// Host side of libep: configuration checks, buffer sizing, the buffer object and
+// the exported C entry points declared in include/ep.h.  Every entry point
+// validates its arguments before touching CUDA and launches nothing on failure.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <new>
+
+#include "ep.h"
+#include "ep_internal.cuh"
+
+struct ep_buffer {
+    ep_config cfg;
+    ep_buffer_ptrs ptrs;
+    ep_buffer_sizes sizes;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+int check_config(const ep_config* c) {
+    if (!c) return EP_ERR_INVALID_ARG;
+    if (c->B < 0 || c->P < 1 || c->E < 1 || c->k < 1 || c->M < 0 || c->d < 1)
+        return EP_ERR_INVALID_ARG;
+    if (c->n_zero < 0 || c->n_copy < 0 || c->n_const < 0) return EP_ERR_INVALID_ARG;
+    if (c->B % c->P != 0 || c->E % c->P != 0) return EP_ERR_INVALID_ARG;
+    if (c->quant_mode != 0 && c->quant_mode != 2) return EP_ERR_INVALID_ARG;
+    if (c->smooth_rows != 0 && c->smooth_rows != 1) return EP_ERR_INVALID_ARG;
+    if (c->layout != 0) return EP_ERR_UNSUPPORTED;
+    if (c->d % 16 != 0) return EP_ERR_INVALID_ARG;
+    if (c->k > ep::kMaxK) return EP_ERR_INVALID_ARG;
+    if (c->d > ep::kMaxD) return EP_ERR_UNSUPPORTED;
+    if (c->E > ep::kMaxE) return EP_ERR_UNSUPPORTED;
+    const long long n_special = (long long)c->n_zero + c->n_copy + c->n_const;
+    if (n_special > ep::kMaxSpecial) return EP_ERR_UNSUPPORTED;
+    if (c->B / c->P > c->M) return EP_ERR_CAPACITY;
+    const long long rows = (long long)c->E * c->P * c->M;
+    if (rows >= (1LL << 31)) return EP_ERR_CAPACITY;
+    if ((long long)c->B * c->k >= (1LL << 31)) return EP_ERR_CAPACITY;
+    return EP_OK;
+}
+
+void fill_sizes(const ep_config* c, ep_buffer_sizes* s) {
+    const size_t E_tot = (size_t)c->E + c->n_zero + c->n_copy + c->n_const;
+    const size_t n_special = (size_t)c->n_zero + c->n_copy + c->n_const;
+    const size_t rows = (size_t)c->E * c->P * c->M;
+    const size_t esz = c->quant_mode == 2 ? 1 : 2;
+    s->expert_count = 4 * E_tot;
+    s->expert_offset = 4 * (E_tot + 1);
+    s->recv_count = 4 * (size_t)c->E * c->P;
+    s->dst_pos = 4 * (size_t)c->B * c->k;
+    s->recv_src = 4 * rows;
+    s->recv_x = rows * (size_t)c->d * esz;
+    s->recv_scale = c->quant_mode == 2 ? 4 * rows : 0;
+    s->token_scale = c->quant_mode == 2 ? 4 * (size_t)c->B : 0;
+    const size_t ws = sizeof(ep::WsHeader) + 4 * (size_t)c->P * n_special;
+    s->workspace = (ws + 255) & ~(size_t)255;
+}
+
+bool ptr_ok(const void* p, size_t size) { return size == 0 || (p != nullptr && aligned16(p)); }
+
+}  // namespace
+
+extern "C" {
+
+int ep_buffer_size(const ep_config* cfg, ep_buffer_sizes* out) {
+    if (!out) return EP_ERR_INVALID_ARG;
+    const int st = check_config(cfg);
+    if (st != EP_OK) return st;
+    fill_sizes(cfg, out);
+    return EP_OK;
+}
+
+int ep_buffer_create(const ep_config* cfg, const ep_buffer_ptrs* ptrs, ep_buffer** out) {
+    if (!out || !ptrs) return EP_ERR_INVALID_ARG;
+    *out = nullptr;
+    const int st = check_config(cfg);
+    if (st != EP_OK) return st;
+    ep_buffer_sizes s;
+    fill_sizes(cfg, &s);
+    if (!ptr_ok(ptrs->expert_count, s.expert_count) || !ptr_ok(ptrs->expert_offset, s.expert_offset) ||
+        !ptr_ok(ptrs->recv_count, s.recv_count) || !ptr_ok(ptrs->dst_pos, s.dst_pos) ||
+        !ptr_ok(ptrs->recv_src, s.recv_src) || !ptr_ok(ptrs->recv_x, s.recv_x) ||
+        !ptr_ok(ptrs->recv_scale, s.recv_scale) || !ptr_ok(ptrs->token_scale, s.token_scale) ||
+        !ptr_ok(ptrs->workspace, s.workspace))
+        return EP_ERR_INVALID_ARG;
+    if (cudaMemset(ptrs->workspace, 0, s.workspace) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return EP_ERR_CUDA;
+    ep_buffer* b = new (std::nothrow) ep_buffer;
+    if (!b) return EP_ERR_INVALID_ARG;
+    b->cfg = *cfg;
+    b->ptrs = *ptrs;
+    b->sizes = s;
+    *out = b;
+    return EP_OK;
+}
+
+int ep_buffer_destroy(ep_buffer* buf) {
+    delete buf;
+    return EP_OK;
+}
+
+int ep_layout(ep_buffer* buf, const int32_t* topk_idx, ep_stream_t stream) {
+    if (!buf) return EP_ERR_INVALID_ARG;
+    if (buf->cfg.B > 0 && (!topk_idx || !aligned4(topk_idx))) return EP_ERR_INVALID_ARG;
+    return ep::launch_layout(ep::make_shape(buf->cfg), buf->ptrs, topk_idx,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale, ep_stream_t stream) {
+    if (!buf) return EP_ERR_INVALID_ARG;
+    const ep_config& c = buf->cfg;
+    if (c.B > 0 && (!x || !aligned16(x))) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && (c.smooth_rows == 0 || !aligned16(smooth_scale))) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && c.quant_mode != 2) return EP_ERR_INVALID_ARG;
+    return ep::launch_dispatch(ep::make_shape(c), buf->ptrs, x, smooth_scale,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,
+               const float* topk_weights, const uint16_t* ori_x, const uint16_t* a1,
+               const uint16_t* a2, const uint16_t* v, uint16_t* y, ep_stream_t stream) {
+    if (!buf) return EP_ERR_INVALID_ARG;
+    const ep_config& c = buf->cfg;
+    if (c.B > 0) {
+        if (!expert_out || !aligned16(expert_out)) return EP_ERR_INVALID_ARG;
+        if (!topk_idx || !aligned4(topk_idx) || !topk_weights || !aligned4(topk_weights))
+            return EP_ERR_INVALID_ARG;
+        if (!y || !aligned16(y)) return EP_ERR_INVALID_ARG;
+        if (c.n_copy + c.n_const > 0 && (!ori_x || !aligned16(ori_x))) return EP_ERR_INVALID_ARG;
+        if (c.n_const > 0 && (!a1 || !a2 || !v || !aligned16(a1) || !aligned16(a2) || !aligned16(v)))
+            return EP_ERR_INVALID_ARG;
+        if (y == ori_x || y == expert_out) return EP_ERR_INVALID_ARG;
+    }
+    return ep::launch_combine(ep::make_shape(c), buf->ptrs, expert_out, topk_idx, topk_weights,
+                              ori_x, a1, a2, v, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ep_buffer_check(ep_buffer* buf, ep_stream_t stream, uint32_t* err_bits) {
+    if (!buf || !err_bits) return EP_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    auto* hdr = reinterpret_cast<ep::WsHeader*>(buf->ptrs.workspace);
+    unsigned host = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaMemcpy(&host, &hdr->err, sizeof host, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return EP_ERR_CUDA;
+    if (cudaMemset(&hdr->err, 0, sizeof host) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return EP_ERR_CUDA;
+    *err_bits = host;
+    return EP_OK;
+}
+
+const char* ep_status_str(int status) {
+    switch (status) {
+        case EP_OK: return "ok";
+        case EP_ERR_INVALID_ARG: return "invalid argument";
+        case EP_ERR_UNSUPPORTED: return "unsupported configuration";
+        case EP_ERR_CAPACITY: return "capacity exceeded (T > M or row ids overflow int32)";
+        case EP_ERR_CUDA: return "CUDA error";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,131 @@
+// Internal declarations shared by the libep translation units (host launchers,
+// the buffer object, device helpers).  Not part of the public ABI (include/ep.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ep.h"
+
+namespace ep {
+
+// Workspace header at the start of the caller's workspace array.  The layout
+// kernel's per-rank special-expert partial counts follow it.
+struct WsHeader {
+    unsigned int done;  // CTAs of the current layout launch that have finished
+    unsigned int err;   // device error word (EP_ERRBIT_*)
+    unsigned int pad[62];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
+
+constexpr int kMaxE = 2048;        // routed experts (Ascend: local_expert_num * ranks <= 2048)
+constexpr int kMaxSpecial = 2048;  // zero + copy + const experts
+constexpr int kMaxK = 16;          // picks per token (Ascend: 0 < K <= 16)
+constexpr int kMaxD = 32768;     // 256 threads x 8 units of 16 elements
+
+struct Shape {
+    int B, d, k, P, M, E, Z, C, K, T, L, E_tot, n_special;
+    int quant_mode;
+    long long rows;  // E * P * M receive rows
+};
+
+inline Shape make_shape(const ep_config& c) {
+    Shape s;
+    s.B = c.B; s.d = c.d; s.k = c.k; s.P = c.P; s.M = c.M; s.E = c.E;
+    s.Z = c.n_zero; s.C = c.n_copy; s.K = c.n_const;
+    s.T = c.B / c.P;
+    s.L = c.E / c.P;
+    s.n_special = c.n_zero + c.n_copy + c.n_const;
+    s.E_tot = c.E + s.n_special;
+    s.quant_mode = c.quant_mode;
+    s.rows = (long long)c.E * c.P * c.M;
+    return s;
+}
+
+// Host launchers (one per kernel family); each returns an EP_* status.
+int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
+                  cudaStream_t stream);
+int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
+                    const float* smooth, cudaStream_t stream);
+int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
+                   const int32_t* topk_idx, const float* topk_weights, const uint16_t* ori_x,
+                   const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
+                   cudaStream_t stream);
+
+// Launch with programmatic dependent launch enabled: the kernel may begin while
+// the previous kernel on the stream drains; every kernel here executes
+// griddepcontrol.wait before it touches memory a predecessor may still use.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+}  // namespace ep
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+#ifdef __CUDACC__
+
+namespace ep {
+
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// 16-byte streaming load through the non-coherent path, not kept in L1.
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// bf16 bits <-> fp32: a bf16 is the high half of a binary32.
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two fp32 -> packed bf16x2, round to nearest even (cvt.rn.bf16x2.f32; NaN stays NaN).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// OR `bits` into the device error word, one atomic per group of converged lanes.
+__device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
+    const unsigned active = __activemask();
+    const unsigned all = __reduce_or_sync(active, bits);
+    if (all && (int)(threadIdx.x & 31) == __ffs(active) - 1) atomicOr(err_word, all);
+}
+
+}  // namespace ep
+
+#endif  // __CUDACC__

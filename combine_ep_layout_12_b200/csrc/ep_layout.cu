@@ -1,0 +1,244 @@
+// Routing layout kernel.
+//
+// Computes, from topk_idx[B][k], the per-expert counts, the per-(expert, source
+// rank) counts, their exclusive prefix and the low-latency receive row of every
+// routed pick (Ascend CANN "low_latency_dispatch": Formula, the alltoallv of the
+// quantized rows; Constraints, the row bound A >= M * P * min(L, K) and the
+// deterministic computation).  Expert g lives on rank g / (E / P) (DeepEP issue
+// #84, masking experiment); id -1 sends nothing.
+//
+// Design.  One CTA per source rank r.  The rank's tokens are processed in rounds
+// of (warps x 32) tokens, one token per lane.  In a round every warp builds, in
+// shared memory, a 32-bit lane mask per routed expert (atomicOr of bit `lane`
+// for each of its token's routed ids).  Because OR is order-independent the
+// masks, and everything derived from them, are deterministic.  An exclusive scan
+// over the warps of popc(mask) per expert, plus the counts of earlier rounds,
+// gives each warp's base; a token's slot inside its (expert, rank) run is then
+//     base[w][g] + popc(mask[w][g] & lanemask_lt)
+// i.e. its rank among rank r's tokens that routed to g, in ascending token order.
+// The last CTA to finish (a ticket counter in the workspace; no CTA ever waits on
+// another) adds the per-rank counts into expert_count and scans expert_offset.
+#include "ep_internal.cuh"
+
+namespace ep {
+namespace {
+
+struct LayoutArgs {
+    const int32_t* topk_idx;
+    int32_t* expert_count;
+    int32_t* expert_offset;
+    int32_t* recv_count;
+    int32_t* dst_pos;
+    int32_t* recv_src;
+    WsHeader* ws;
+    int32_t* sp_partial;  // [P][n_special]
+    int B, k, P, M, E, T, n_special, E_tot;
+    int warps;            // warps per CTA
+};
+
+__global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
+    extern __shared__ unsigned smem[];
+    const int W = a.warps;
+    unsigned* mask = smem;                                         // [W][E]
+    int* pre = reinterpret_cast<int*>(smem + (size_t)W * a.E);     // [W][E]
+    int* run = pre + (size_t)W * a.E;                              // [E] count so far
+    int* spc = run + a.E;                                          // [n_special]
+    __shared__ int s_last;
+
+    const int r = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    for (int g = threadIdx.x; g < E; g += blockDim.x) run[g] = 0;
+    for (int s = threadIdx.x; s < a.n_special; s += blockDim.x) spc[s] = 0;
+
+    unsigned err = 0;
+    const int tok_begin = r * a.T;
+    const int tok_end = tok_begin + a.T;
+    const int per_round = W * 32;
+    unsigned* my_mask = mask + (size_t)warp * E;
+    int* my_pre = pre + (size_t)warp * E;
+
+    for (int round0 = tok_begin; round0 < tok_end; round0 += per_round) {
+        // (1) clear this warp's masks (the previous round's readers of my_mask
+        //     are this warp's own lanes, so a warp barrier suffices)
+        __syncwarp();
+        for (int g = lane; g < E; g += 32) my_mask[g] = 0u;
+        __syncthreads();  // also orders run[] / spc[] init before first use
+
+        const int t = round0 + warp * 32 + lane;
+        const bool valid = t < tok_end;
+        int ids[kMaxK];
+        bool routed[kMaxK];
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+            ids[j] = -1;
+            routed[j] = false;
+            if (j < k && valid) ids[j] = a.topk_idx[(size_t)t * k + j];
+        }
+        // (2) classify; routed ids set their lane bit
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) {
+            if (j >= k || !valid) continue;
+            const int g = ids[j];
+            if (g == -1) continue;
+            if (g < -1 || g >= a.E_tot) {
+                err |= EP_ERRBIT_BAD_ID;
+                continue;
+            }
+            if (g >= E) {
+                atomicAdd(&spc[g - E], 1);
+                continue;
+            }
+            bool dup = false;
+#pragma unroll
+            for (int jj = 0; jj < kMaxK; ++jj)
+                if (jj < j && ids[jj] == g) dup = true;
+            if (dup) {
+                err |= EP_ERRBIT_DUP_ID;
+                continue;
+            }
+            routed[j] = true;
+            atomicOr(&my_mask[g], 1u << lane);
+        }
+        __syncthreads();
+        // (3) per expert: exclusive scan of the warps' popcounts, on top of the
+        //     counts of earlier rounds
+        for (int g = threadIdx.x; g < E; g += blockDim.x) {
+            int c = run[g];
+            for (int w = 0; w < W; ++w) {
+                pre[(size_t)w * E + g] = c;
+                c += __popc(mask[(size_t)w * E + g]);
+            }
+            run[g] = c;
+        }
+        __syncthreads();
+        // (4) slots, receive rows, source map
+        if (valid) {
+            const unsigned lt = lanemask_lt();
+#pragma unroll
+            for (int j = 0; j < kMaxK; ++j) {
+                if (j >= k) continue;
+                int row = -1;
+                if (routed[j]) {
+                    const int g = ids[j];
+                    const int slot = my_pre[g] + __popc(my_mask[g] & lt);
+                    row = g * a.P * a.M + r * a.M + slot;
+                    a.recv_src[row] = t;
+                }
+                a.dst_pos[(size_t)t * k + j] = row;
+            }
+        }
+    }
+    __syncthreads();
+
+    // per-rank outputs
+    for (int g = threadIdx.x; g < E; g += blockDim.x) a.recv_count[(size_t)g * a.P + r] = run[g];
+    for (int s = threadIdx.x; s < a.n_special; s += blockDim.x)
+        a.sp_partial[(size_t)r * a.n_special + s] = spc[s];
+    report_err(&a.ws->err, err);
+
+    // ticket: the last CTA of this launch reduces over ranks
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned ticket = atomicAdd(&a.ws->done, 1u);
+        s_last = (ticket == (unsigned)a.P - 1u);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+
+    // expert_count over all ids, then exclusive prefix into expert_offset.
+    // Thread i owns a contiguous chunk of ids; chunk sums are scanned in smem.
+    int* chunk = reinterpret_cast<int*>(smem);  // reuse: [blockDim]
+    const int n = a.E_tot;
+    const int per = (n + blockDim.x - 1) / blockDim.x;
+    const int lo = min(n, (int)threadIdx.x * per);
+    const int hi = min(n, lo + per);
+    int sum = 0;
+    for (int g = lo; g < hi; ++g) {
+        int c = 0;
+        if (g < E) {
+            for (int q = 0; q < a.P; ++q) c += __ldcg(&a.recv_count[(size_t)g * a.P + q]);
+        } else {
+            for (int q = 0; q < a.P; ++q)
+                c += __ldcg(&a.sp_partial[(size_t)q * a.n_special + (g - E)]);
+        }
+        a.expert_count[g] = c;
+        sum += c;
+    }
+    chunk[threadIdx.x] = sum;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int i = 0; i < (int)blockDim.x; ++i) {
+            const int v = chunk[i];
+            chunk[i] = acc;
+            acc += v;
+        }
+        a.expert_offset[n] = acc;
+        a.ws->done = 0u;  // re-arm the ticket for the next launch
+    }
+    __syncthreads();
+    int acc = chunk[threadIdx.x];
+    for (int g = lo; g < hi; ++g) {
+        a.expert_offset[g] = acc;
+        acc += __ldcg(&a.expert_count[g]);
+    }
+}
+
+}  // namespace
+
+int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
+                  cudaStream_t stream) {
+    if (s.B == 0) {
+        // no tokens: counts are all zero
+        cudaError_t e1 = cudaMemsetAsync(p.expert_count, 0, sizeof(int32_t) * s.E_tot, stream);
+        cudaError_t e2 = cudaMemsetAsync(p.expert_offset, 0, sizeof(int32_t) * (s.E_tot + 1), stream);
+        cudaError_t e3 = cudaMemsetAsync(p.recv_count, 0, sizeof(int32_t) * s.E * s.P, stream);
+        return (e1 || e2 || e3) ? EP_ERR_CUDA : EP_OK;
+    }
+    // warps per CTA: enough for one round of the rank's tokens, at most 32,
+    // within the shared-memory budget (two [warps][E] arrays plus [E] + specials)
+    const size_t budget = 160 * 1024;
+    const size_t fixed = sizeof(int) * ((size_t)s.E + s.n_special);
+    int warps = (s.T + 31) / 32;
+    if (warps > 32) warps = 32;
+    if (warps < 1) warps = 1;
+    while (warps > 1 && fixed + (size_t)warps * s.E * 8 > budget) --warps;
+    size_t smem = fixed + (size_t)warps * s.E * 8;
+    const size_t need_tail = sizeof(int) * (size_t)warps * 32;  // chunk sums of the last CTA
+    if (smem < need_tail) smem = need_tail;
+
+    static bool attr_set[16] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 16 && !attr_set[dev]) {
+        if (cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)budget) != cudaSuccess)
+            return EP_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+
+    LayoutArgs a;
+    a.topk_idx = topk_idx;
+    a.expert_count = p.expert_count;
+    a.expert_offset = p.expert_offset;
+    a.recv_count = p.recv_count;
+    a.dst_pos = p.dst_pos;
+    a.recv_src = p.recv_src;
+    a.ws = reinterpret_cast<WsHeader*>(p.workspace);
+    a.sp_partial = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.workspace) + sizeof(WsHeader));
+    a.B = s.B; a.k = s.k; a.P = s.P; a.M = s.M; a.E = s.E; a.T = s.T;
+    a.n_special = s.n_special; a.E_tot = s.E_tot;
+    a.warps = warps;
+    cudaError_t e = launch_pdl(layout_kernel, dim3(s.P), dim3(warps * 32), smem, stream, a);
+    return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+}  // namespace ep

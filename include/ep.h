@@ -1,0 +1,186 @@
+/*
+ * ep.h -- C ABI of libep: MoE expert-parallel token dispatch and combine on one
+ * B200, with the EP ranks as logical partitions of the GPU's memory.
+ *
+ * The operation (sources: Ascend CANN page "low_latency_dispatch", sections
+ * Function / Formula, Constraints and Example; DeepEP issue #84 "Profiling
+ * dispatch_t for low-latency kernel dispatch bandwidth"):
+ *
+ *   B tokens x[B][d] (bf16) are split over P logical ranks, T = B / P tokens each;
+ *   token t belongs to source rank r = t / T.  Each token picks k experts
+ *   topk_idx[t][j].  Routed experts are ids [0, E); expert g lives on rank g / L,
+ *   L = E / P (DeepEP issue #84, masking experiment).  Ids E .. E+Z-1 are zero
+ *   experts, then C copy experts, then K constant experts (Ascend Example:
+ *   num_experts = 32 with one zero and one copy expert uses ids 32 and 33).
+ *   Id -1 means "not routed" (DeepEP issue #84 masks picks with -1).
+ *
+ *   ep_layout   counts per expert and per (expert, source rank), their exclusive
+ *               prefix, the receive row of every routed pick and the source token
+ *               of every receive row.  Receive layout is the low-latency one:
+ *               row = g * P * M + r * M + slot, i.e. a [E][P*M][d] buffer that
+ *               rank q reads as [L][P*M][d] starting at expert q*L.  slot is the
+ *               rank of token t among rank r's tokens that routed to g, ascending
+ *               t (the page states the computation is deterministic).
+ *   ep_dispatch quant_mode 0: expand_x row = x[t] (bf16 bits copied).
+ *               quant_mode 2: xf = fp32(x) * smooth_scale, s = 127 / max|xf| over
+ *               the row, q = CastToInt8(xf * s) (round half to even, saturate),
+ *               inv = 1 / s; q goes to every receive row of t and inv to
+ *               recv_scale of those rows and to token_scale[t]
+ *               (Ascend Formula, dynamic quantization scenario).
+ *   ep_combine  y[t] = bf16( sum_j w[t][j] * e(t,j) ), fp32 fused multiply-add in
+ *               pick order j from 0, rounded once to bf16 (nearest even), where
+ *               e(t,j) = expert_out[dst_pos[t][j]] for a routed pick, ori_x[t]
+ *               for a copy expert, a1[c] * ori_x[t] + a2[c] * v[c] (fp32) for
+ *               constant expert c, and the term is skipped for -1 and zero
+ *               experts (Ascend Formula, special expert scenario).
+ *
+ * Conventions for every entry point:
+ *  - All device pointers are owned by the caller (e.g. torch tensors).  The
+ *    library never allocates or frees device memory; ep_buffer_create allocates
+ *    one small host struct.
+ *  - bf16 values travel as their uint16_t bit patterns.  Arrays are dense,
+ *    row-major, with the shapes given below.  Pointers to bf16/int8 row data
+ *    must be 16-byte aligned (d % 16 == 0 keeps every row aligned).
+ *  - Launching calls are asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and return after the launch.  Host-side validation
+ *    failures return a negative status and launch nothing.  Bad routing data
+ *    found on the device (ids outside [-1, E+Z+C+K), a routed id repeated inside
+ *    a token) does not trap: the pick is dropped and a bit is set in the buffer's
+ *    device error word, read by ep_buffer_check.
+ *  - The device that runs the kernels is the one current on the calling thread
+ *    (the CUDA context current when the call is made).
+ */
+#ifndef EP_H
+#define EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols keep default visibility even when the library is built with
+ * -fvisibility=hidden. */
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* ep_stream_t;
+
+/* Status codes. */
+#define EP_OK 0
+#define EP_ERR_INVALID_ARG (-1) /* null or misaligned pointer, bad config field */
+#define EP_ERR_UNSUPPORTED (-2) /* well-formed but outside what this build supports */
+#define EP_ERR_CAPACITY (-3)    /* T > M, or int32 row ids would overflow */
+#define EP_ERR_CUDA (-4)        /* a CUDA runtime call or a launch failed */
+
+/* Bits of the device error word. */
+#define EP_ERRBIT_BAD_ID 0x1u /* an id < -1 or >= E+Z+C+K: that pick was dropped */
+#define EP_ERRBIT_DUP_ID 0x2u /* a routed id repeated in one token: later copies dropped */
+#define EP_ERRBIT_ROW_RANGE 0x4u /* a dst_pos outside [-1, E*P*M) reached dispatch or
+                                    combine (e.g. no ep_layout ran): that pick was skipped */
+
+/*
+ * Problem description.  Constraints checked by ep_buffer_size/ep_buffer_create:
+ *   B >= 0, P >= 1, B % P == 0, E >= 1, E % P == 0 (Ascend Example: num_experts must
+ *   be a multiple of the MoE rank count), E <= 2048 (Constraints:
+ *   local_expert_num * ep_world_size <= 2048), 1 <= k <= 16 (Constraints:
+ *   0 < K <= 16), T = B / P <= M, Z, C, K >= 0 with Z + C + K <= 2048,
+ *   E*P*M < 2^31 (int32 row ids), 16 <= d <= 32768 with d % 16 == 0,
+ *   quant_mode in {0, 2}, smooth_rows in {0, 1}, layout == 0.
+ */
+typedef struct {
+    int32_t B;           /* tokens over all logical ranks */
+    int32_t d;           /* hidden size */
+    int32_t k;           /* picks per token */
+    int32_t P;           /* logical EP ranks */
+    int32_t M;           /* max tokens per rank (rows per (expert, source rank)) */
+    int32_t E;           /* routed experts */
+    int32_t n_zero;      /* zero experts  (ids E .. E+Z-1) */
+    int32_t n_copy;      /* copy experts  (next C ids) */
+    int32_t n_const;     /* constant experts (next K ids) */
+    int32_t quant_mode;  /* 0: bf16 pass-through; 2: dynamic per-token int8 */
+    int32_t smooth_rows; /* 0: no smooth scale; 1: one fp32 [d] vector may be given */
+    int32_t layout;      /* 0: low-latency [E][P*M][d] receive layout */
+} ep_config;
+
+/* Byte sizes of the caller-allocated device arrays (0 = not needed). */
+typedef struct {
+    size_t expert_count;  /* int32 [E+Z+C+K]    picks per expert id */
+    size_t expert_offset; /* int32 [E+Z+C+K+1]  exclusive prefix of expert_count */
+    size_t recv_count;    /* int32 [E][P]       rows of expert g from source rank r
+                             (per receiving rank q: [L][P] = ep_recv_counts) */
+    size_t dst_pos;       /* int32 [B][k]       receive row of each pick, -1 if none */
+    size_t recv_src;      /* int32 [E*P*M]      source token of each receive row
+                             (the combine's source map); rows past a run's count
+                             are not written */
+    size_t recv_x;        /* [E*P*M][d] int8 (quant_mode 2) or bf16 (quant_mode 0) */
+    size_t recv_scale;    /* fp32 [E*P*M]       1/s of the row's token (quant_mode 2) */
+    size_t token_scale;   /* fp32 [B]           1/s per token (quant_mode 2) */
+    size_t workspace;     /* scratch words; zero-filled by ep_buffer_create */
+} ep_buffer_sizes;
+
+/* Device pointers matching ep_buffer_sizes (NULL where the size is 0). */
+typedef struct {
+    int32_t* expert_count;
+    int32_t* expert_offset;
+    int32_t* recv_count;
+    int32_t* dst_pos;
+    int32_t* recv_src;
+    void* recv_x;
+    float* recv_scale;
+    float* token_scale;
+    void* workspace;
+} ep_buffer_ptrs;
+
+typedef struct ep_buffer ep_buffer;
+
+/* Validate `cfg` and report the byte size of every array.  Host only, no CUDA call.
+ * Returns EP_OK, EP_ERR_INVALID_ARG, EP_ERR_UNSUPPORTED or EP_ERR_CAPACITY. */
+EP_API int ep_buffer_size(const ep_config* cfg, ep_buffer_sizes* out);
+
+/* Wrap caller memory into a buffer object (a host struct; no device allocation).
+ * Every pointer whose size is non-zero must be non-NULL and 16-byte aligned.
+ * Zero-fills the workspace with a synchronous cudaMemset on the current device.
+ * On success *out owns the host struct until ep_buffer_destroy. */
+EP_API int ep_buffer_create(const ep_config* cfg, const ep_buffer_ptrs* ptrs, ep_buffer** out);
+
+/* Free the host struct.  Device memory stays with the caller.  NULL is accepted. */
+EP_API int ep_buffer_destroy(ep_buffer* buf);
+
+/* Routing layout from topk_idx (int32 [B][k], device).  Writes expert_count,
+ * expert_offset, recv_count, dst_pos and the written rows of recv_src. */
+EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, ep_stream_t stream);
+
+/* Quantize (quant_mode 2) or pass through (0) x (bf16 [B][d], device) and scatter
+ * every routed pick into recv_x (plus recv_scale, token_scale in mode 2), using
+ * the dst_pos of the latest ep_layout on this buffer.  smooth_scale is an fp32
+ * [d] device vector or NULL; it must be NULL when cfg.smooth_rows == 0. */
+EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale,
+                ep_stream_t stream);
+
+/* Weighted combine into y (bf16 [B][d], device).  expert_out: bf16 [E*P*M][d]
+ * receive-layout expert outputs (may alias recv_x when quant_mode is 0);
+ * topk_idx int32 [B][k] and topk_weights fp32 [B][k] as given to ep_layout;
+ * ori_x bf16 [B][d] (required when C + K > 0, else may be NULL);
+ * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos.
+ * y must not overlap any input. */
+EP_API int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,
+               const float* topk_weights, const uint16_t* ori_x, const uint16_t* a1,
+               const uint16_t* a2, const uint16_t* v, uint16_t* y, ep_stream_t stream);
+
+/* Synchronize `stream`, read the device error word into *err_bits and clear it. */
+EP_API int ep_buffer_check(ep_buffer* buf, ep_stream_t stream, uint32_t* err_bits);
+
+/* Static text for a status code. */
+EP_API const char* ep_status_str(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EP_H */

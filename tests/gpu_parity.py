@@ -1,0 +1,147 @@
+"""Parity harness: run libep on the GPU and compare with the CPU oracle.
+
+Expected values come only from the oracle (or from the seeded input generators);
+nothing the GPU computes is fed back into the oracle.  Expert outputs for the
+combine check are drawn by the seeded generator and placed at the receive rows
+the oracle's layout names, so the GPU combine reads them through its own
+dst_pos.
+"""
+import numpy as np
+import torch
+
+import oracle
+from combine_ep_layout_12_b200 import runner
+from combine_ep_layout_12_b200 import workloads as wl
+
+COMBINE_REL_TOL = 8e-3
+
+
+def ocfg(w, B=None, P=None, M=None):
+    return oracle.make_cfg(w.B if B is None else B, w.d, w.k, w.P if P is None else P,
+                           w.M if M is None else M, w.E, w.n_zero, w.n_copy, w.n_const,
+                           w.quant_mode)
+
+
+def bf16_to_f32(bits):
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+class Report:
+    def __init__(self):
+        self.fails = []
+        self.notes = {}
+
+    def check(self, cond, msg):
+        if not cond:
+            self.fails.append(msg)
+
+    def assert_ok(self):
+        assert not self.fails, "\n".join(self.fails)
+
+
+def check_layout(rep, w, pipe, ref):
+    buf = pipe.buf
+    rep.check(np.array_equal(buf.expert_count.cpu().numpy(), ref["expert_count"]),
+              "%s: expert_count differs" % w.name)
+    rep.check(np.array_equal(buf.expert_offset.cpu().numpy(), ref["expert_offset"]),
+              "%s: expert_offset differs" % w.name)
+    rep.check(np.array_equal(buf.recv_count.cpu().numpy(), ref["recv_count"]),
+              "%s: recv_count differs" % w.name)
+    dp = buf.dst_pos.cpu().numpy()
+    rep.check(np.array_equal(dp, ref["dst_pos"]), "%s: dst_pos differs (%d picks)"
+              % (w.name, int((dp != ref["dst_pos"]).sum())))
+    rows = np.nonzero(ref["recv_src"] >= 0)[0]
+    got = buf.recv_src[torch.from_numpy(rows).to(buf.device)].cpu().numpy()
+    rep.check(np.array_equal(got, ref["recv_src"][rows]), "%s: recv_src differs" % w.name)
+
+
+def check_dispatch(rep, w, pipe, inp, ref_lay, sample_picks=None, rng=None):
+    """quant_out / scales of the oracle vs the GPU receive rows of routed picks."""
+    cfg = ocfg(w)
+    q, ts = oracle.quantize(cfg, inp["x"], inp["smooth"])
+    dp = ref_lay["dst_pos"]
+    tt, jj = np.nonzero(dp >= 0)
+    if sample_picks is not None and tt.size > sample_picks:
+        sel = (rng or np.random.default_rng(0)).choice(tt.size, sample_picks, replace=False)
+        sel.sort()
+        tt, jj = tt[sel], jj[sel]
+    rows = dp[tt, jj]
+    buf = pipe.buf
+    rows_d = torch.from_numpy(rows.astype(np.int64)).to(buf.device)
+    got = buf.recv_x[rows_d]
+    if w.quant_mode == 2:
+        got = got.cpu().numpy()
+        bad = np.nonzero(np.any(got != q[tt], axis=1))[0]
+        rep.check(bad.size == 0, "%s: int8 payload differs in %d of %d rows" % (w.name, bad.size, rows.size))
+        gs = buf.recv_scale[rows_d].cpu().numpy()
+        rep.check(np.array_equal(gs.view(np.uint32), ts[tt].view(np.uint32)),
+                  "%s: recv_scale differs" % w.name)
+        gts = buf.token_scale.cpu().numpy()
+        rep.check(np.array_equal(gts.view(np.uint32), ts.view(np.uint32)),
+                  "%s: token_scale differs in %d tokens" % (w.name, int((gts != ts).sum())))
+    else:
+        got = runner.bf16_bits(got)
+        bad = np.nonzero(np.any(got != q[tt], axis=1))[0]
+        rep.check(bad.size == 0, "%s: bf16 payload differs in %d of %d rows" % (w.name, bad.size, rows.size))
+    rep.notes["dispatch_rows_checked"] = int(rows.size)
+    return q, ts
+
+
+def place_expert_rows(w, pipe, ref_lay, tokens, seed_offset=0):
+    """Draw expert outputs for every routed pick of `tokens`, write them to the GPU
+    expert_out at the oracle's rows; return the compact rows and compact dst_pos."""
+    dp = ref_lay["dst_pos"][tokens]
+    routed = dp >= 0
+    n = int(routed.sum())
+    vals = wl.gen_expert_rows(w, max(n, 1), seed_offset)[:n]
+    compact = np.full(dp.shape, -1, np.int32)
+    compact[routed] = np.arange(n, dtype=np.int32)
+    if n:
+        rows_d = torch.from_numpy(dp[routed].astype(np.int64)).to(pipe.device)
+        pipe.expert_out[rows_d] = runner.bf16_tensor(vals, pipe.device)
+    return vals, compact
+
+
+def check_combine(rep, w, pipe, inp, dev_inp, ref_lay, tokens=None, seed_offset=0, run=True):
+    if tokens is None:
+        tokens = np.arange(w.B)
+    vals, compact = place_expert_rows(w, pipe, ref_lay, tokens, seed_offset)
+    if run:
+        torch.cuda.synchronize()
+        pipe.combine(dev_inp)
+    y_gpu = runner.bf16_bits(pipe.y[torch.from_numpy(tokens).to(pipe.device)])
+    sub = ocfg(w, B=len(tokens), P=1, M=max(len(tokens), 1))
+    idx = inp["topk_idx"][tokens]
+    wts = inp["topk_weights"][tokens]
+    x = inp["x"][tokens]
+    y_ref = oracle.combine(sub, vals if vals.shape[0] else None, idx, wts, compact, x,
+                           inp["a1"], inp["a2"], inp["v"])
+    compare_combine(rep, w.name, y_gpu, y_ref, idx, wts, compact, vals, x, w)
+
+
+def compare_combine(rep, name, y_gpu, y_ref, idx, wts, compact, vals, x, w):
+    exact = y_gpu == y_ref
+    n_diff = int((~exact).sum())
+    rep.notes["combine_elements"] = int(exact.size)
+    rep.notes["combine_not_bitexact"] = n_diff
+    if n_diff == 0:
+        return
+    # tolerance: |d| <= 8e-3 |y_ref|  or  |d| <= 2^-8 * sum_j |w_j e_j|
+    g = bf16_to_f32(y_gpu).astype(np.float64)
+    r = bf16_to_f32(y_ref).astype(np.float64)
+    mag = np.zeros_like(r)
+    E, Z, C = w.E, w.n_zero, w.n_copy
+    xf = bf16_to_f32(x).astype(np.float64)
+    for j in range(idx.shape[1]):
+        gsel = idx[:, j]
+        e = np.zeros_like(r)
+        routed = compact[:, j] >= 0
+        if routed.any():
+            e[routed] = bf16_to_f32(vals[compact[routed, j]])
+        cp = (gsel >= E + Z) & (gsel < E + Z + C)
+        e[cp] = xf[cp]
+        mag += np.abs(wts[:, j:j + 1].astype(np.float64) * e)
+    ok = (np.abs(g - r) <= COMBINE_REL_TOL * np.abs(r)) | (np.abs(g - r) <= 2.0**-8 * mag)
+    rep.check(bool(ok.all()), "%s: combine outside tolerance at %d elements" % (name, int((~ok).sum())))
+    rep.check(n_diff == 0, "%s: combine not bit-exact at %d elements (within tolerance: %s)"
+              % (name, n_diff, bool(ok.all())))

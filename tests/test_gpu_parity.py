@@ -1,0 +1,311 @@
+"""GPU parity: libep (through the C ABI) against the CPU oracle on the named
+workloads and on edge cases.  Layout, source maps, int8/bf16 payloads and scales
+must be bit-exact; combine must be within 8e-3 relative (one bf16 ulp of the
+accumulated magnitude near zero) and, with the same fused multiply-add order on
+both sides, is also required to be bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from combine_ep_layout_12_b200 import EPBuffer, runner
+from combine_ep_layout_12_b200 import workloads as wl
+from combine_ep_layout_12_b200 import build as ep_build
+from tests import gpu_parity as gp
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="session")
+def dev():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    ep_build.build()
+    torch.cuda.set_device(0)
+    return torch.device("cuda", 0)
+
+
+def free_bytes():
+    torch.cuda.empty_cache()
+    return torch.cuda.mem_get_info()[0]
+
+
+def need_bytes(w, separate_expert_out):
+    rows = w.rows
+    esz = 1 if w.quant_mode == 2 else 2
+    total = rows * w.d * esz + rows * 4 * (3 if w.quant_mode == 2 else 1)
+    if separate_expert_out:
+        total += rows * w.d * 2
+    total += 2 * w.B * w.d * 2 + 16 * w.B * w.k
+    return total
+
+
+def full_check(w, dev, inp=None, tokens=None, sample_picks=None, separate=True):
+    """Layout + dispatch + combine of one workload against the oracle."""
+    inp = inp if inp is not None else wl.generate(w)
+    if need_bytes(w, separate) > free_bytes() - (4 << 30):
+        pytest.skip("%s needs %.1f GB of device memory" % (w.name, need_bytes(w, separate) / 1e9))
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev, alias_expert_out=not separate)
+    rep = gp.Report()
+    pipe.layout(dev_inp)
+    pipe.dispatch(dev_inp)
+    err = pipe.buf.check()
+    ref = oracle.layout(gp.ocfg(w), inp["topk_idx"])
+    rep.check(err == ref["err"], "%s: device error bits %#x, oracle %#x" % (w.name, err, ref["err"]))
+    gp.check_layout(rep, w, pipe, ref)
+    gp.check_dispatch(rep, w, pipe, inp, ref, sample_picks=sample_picks)
+    gp.check_combine(rep, w, pipe, inp, dev_inp, ref, tokens=tokens)
+    err = pipe.buf.check()
+    rep.check(err == 0, "%s: error bits after combine %#x" % (w.name, err))
+    rep.assert_ok()
+    return pipe, dev_inp, inp, ref
+
+
+# ----------------------------------------------------------------------------- named workloads
+
+
+@pytest.mark.parametrize("name", ["tiny_q0", "tiny_q2"])
+def test_tiny(dev, name):
+    full_check(wl.get(name), dev)
+
+
+def test_tiny_q2_random_smooth(dev):
+    full_check(wl.get("tiny_q2").with_(name="tiny_q2_rand_smooth", smooth="rand", seed=3), dev)
+
+
+def test_decode(dev):
+    """DeepSeek-V3-shaped decode in the launch configuration the benchmark times."""
+    full_check(wl.get("decode"), dev)
+
+
+def test_skewed_specials(dev):
+    full_check(wl.get("skewed"), dev)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 64, 256])
+@pytest.mark.parametrize("qm", [0, 2])
+def test_sweep_small(dev, T, qm):
+    full_check(wl.get("sweep_T%d_q%d" % (T, qm)), dev)
+
+
+@pytest.mark.parametrize("qm", [0, 2])
+def test_sweep_T1024_sampled(dev, qm):
+    w = wl.get("sweep_T1024_q%d" % qm)
+    rng = np.random.default_rng(1024)
+    tokens = np.sort(rng.choice(w.B, 512, replace=False))
+    full_check(w, dev, tokens=tokens, sample_picks=8192, separate=(qm == 2))
+
+
+def test_sweep_T4096_q2_sampled(dev):
+    """120 GB int8 receive buffer; combine is checked through the mode-0 aliasing
+    path of the bf16 workloads (a bf16 expert_out of this shape is 240 GB)."""
+    w = wl.get("sweep_T4096_q2")
+    if need_bytes(w, False) > free_bytes() - (4 << 30):
+        pytest.skip("needs %.1f GB" % (need_bytes(w, False) / 1e9))
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    buf = EPBuffer(w, device=dev)
+    buf.layout(dev_inp["topk_idx"])
+    buf.dispatch(dev_inp["x"])
+    rep = gp.Report()
+    ref = oracle.layout(gp.ocfg(w), inp["topk_idx"])
+    err = buf.check()
+    rep.check(err == ref["err"], "error bits")
+
+    class P:
+        pass
+    pipe = P()
+    pipe.buf = buf
+    gp.check_layout(rep, w, pipe, ref)
+    gp.check_dispatch(rep, w, pipe, inp, ref, sample_picks=8192)
+    rep.assert_ok()
+
+
+def test_prefill(dev):
+    """High-throughput prefill, bf16 payload, 120 GB low-latency buffer.  Layout
+    bit-exact in full, payload on sampled picks, combine(dispatch(x)) == x with
+    one-hot weights in full, and combine against the oracle on sampled tokens."""
+    w = wl.get("prefill")
+    if need_bytes(w, False) > free_bytes() - (4 << 30):
+        pytest.skip("needs %.1f GB" % (need_bytes(w, False) / 1e9))
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev, alias_expert_out=True)
+    rep = gp.Report()
+    pipe.layout(dev_inp)
+    pipe.dispatch(dev_inp)
+    ref = oracle.layout(gp.ocfg(w), inp["topk_idx"])
+    rep.check(pipe.buf.check() == ref["err"], "error bits")
+    gp.check_layout(rep, w, pipe, ref)
+    gp.check_dispatch(rep, w, pipe, inp, ref, sample_picks=16384)
+    # identity expert + one-hot weights: y == x bitwise, every token
+    rng = np.random.default_rng(77)
+    onehot = np.zeros((w.B, w.k), np.float32)
+    onehot[np.arange(w.B), rng.integers(0, w.k, w.B)] = 1.0
+    dev1 = dict(dev_inp)
+    dev1["topk_weights"] = torch.from_numpy(onehot).to(dev)
+    y = pipe.combine(dev1)
+    rep.check(torch.equal(y.view(torch.int16), dev_inp["x"].view(torch.int16)),
+              "prefill: combine(dispatch(x)) != x with one-hot weights")
+    # sampled tokens against the oracle with softmax weights
+    tokens = np.sort(rng.choice(w.B, 512, replace=False))
+    gp.check_combine(rep, w, pipe, inp, dev_inp, ref, tokens=tokens)
+    rep.assert_ok()
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+
+def small(name, **kw):
+    base = dict(B=96, d=128, k=4, P=4, M=24, E=16, quant_mode=2)
+    base.update(kw)
+    return wl.Workload(name, **base)
+
+
+def test_empty_batch(dev):
+    w = small("empty", B=0)
+    buf = EPBuffer(w, device=dev)
+    idx = torch.empty((0, w.k), dtype=torch.int32, device=dev)
+    x = torch.empty((0, w.d), dtype=torch.bfloat16, device=dev)
+    wts = torch.empty((0, w.k), dtype=torch.float32, device=dev)
+    eo = torch.zeros((w.rows, w.d), dtype=torch.bfloat16, device=dev)
+    buf.layout(idx)
+    buf.dispatch(x)
+    y = buf.combine(eo, idx, wts, ori_x=x)
+    assert buf.check() == 0
+    assert y.shape == (0, w.d)
+    assert int(buf.expert_count.sum()) == 0 and int(buf.expert_offset[-1]) == 0
+    assert int(buf.recv_count.abs().sum()) == 0
+
+
+def test_ragged_dirty_specials(dev):
+    """T = 37 (not a warp multiple), d = 272 (17 int8 units), 3 ranks, special
+    experts, smooth scale, -1 picks, out-of-range ids and a duplicate id."""
+    w = wl.Workload("ragged", B=111, d=272, k=3, P=3, M=40, E=9, n_zero=1, n_copy=1, n_const=1,
+                    quant_mode=2, smooth="rand", seed=5)
+    inp = wl.generate(w)
+    rng = np.random.default_rng(5)
+    idx = np.stack([rng.permutation(w.E_tot)[:w.k] for _ in range(w.B)]).astype(np.int32)
+    idx[3, 1] = -1
+    idx[7, 0] = w.E_tot + 2      # not an expert id
+    idx[8, 2] = -9               # not an expert id
+    idx[10] = [4, 5, 4]          # routed id 4 twice: the second copy is dropped
+    inp["topk_idx"] = idx
+    # errors are expected here, so run the steps by hand
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev, alias_expert_out=False)
+    pipe.layout(dev_inp)
+    pipe.dispatch(dev_inp)
+    err = pipe.buf.check()
+    ref = oracle.layout(gp.ocfg(w), idx)
+    assert ref["err"] == (oracle.ERR_BAD_ID | oracle.ERR_DUP_ID)
+    assert err == ref["err"]
+    rep = gp.Report()
+    gp.check_layout(rep, w, pipe, ref)
+    gp.check_dispatch(rep, w, pipe, inp, ref)
+    gp.check_combine(rep, w, pipe, inp, dev_inp, ref)
+    rep.assert_ok()
+
+
+@pytest.mark.parametrize("k,E,P", [(1, 8, 2), (16, 32, 2), (16, 64, 8)])
+def test_k_extremes(dev, k, E, P):
+    w = wl.Workload("k%d" % k, B=P * 40, d=64, k=k, P=P, M=48, E=E, quant_mode=2, seed=k)
+    full_check(w, dev)
+
+
+def test_max_experts(dev):
+    """E = 2048 (the pages' cap on local_expert_num * ranks): the layout kernel
+    runs with fewer warps per CTA (shared-memory budget) and several rounds."""
+    w = wl.Workload("e2048", B=8 * 600, d=64, k=8, P=8, M=600, E=2048, quant_mode=0, seed=11)
+    full_check(w, dev)
+
+
+def test_many_rounds(dev):
+    """2500 tokens per rank: the layout kernel loops over three rounds of 1024."""
+    w = wl.Workload("rounds", B=2 * 2500, d=32, k=6, P=2, M=2600, E=64, quant_mode=2, seed=12)
+    full_check(w, dev)
+
+
+@pytest.mark.parametrize("d", [16, 32768])
+def test_d_extremes(dev, d):
+    w = wl.Workload("d%d" % d, B=32, d=d, k=2, P=2, M=16, E=8, quant_mode=2, seed=d)
+    full_check(w, dev)
+    full_check(w.with_(quant_mode=0, name="d%d_q0" % d), dev)
+
+
+def test_degenerate_rows(dev):
+    """All-zero rows and rows whose 127/amax overflows give q = 0 and scale 0."""
+    w = small("degenerate")
+    inp = wl.generate(w)
+    inp["x"][0] = 0
+    inp["x"][5] = 0x0080          # 2^-126 in every element: 127/amax overflows fp32
+    inp["x"][6, :] = 0
+    inp["x"][6, 3] = 0x8001       # a single negative subnormal
+    full_check(w, dev, inp=inp)
+
+
+def test_all_specials(dev):
+    """Copy experts with dyadic weights give x; zero experts and -1 give +0."""
+    w = small("specials", n_zero=1, n_copy=1, n_const=1, quant_mode=0)
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev)
+    idx = np.full((w.B, w.k), w.E + 1, np.int32)              # copy expert everywhere
+    wts = np.tile(np.array([0.5, 0.25, 0.125, 0.125], np.float32), (w.B, 1))
+    dev_inp["topk_idx"] = torch.from_numpy(idx).to(dev)
+    dev_inp["topk_weights"] = torch.from_numpy(wts).to(dev)
+    y = pipe.step(dev_inp)
+    assert torch.equal(y.view(torch.int16), dev_inp["x"].view(torch.int16))
+    idx[:] = w.E                                               # zero expert
+    idx[:, 1] = -1
+    dev_inp["topk_idx"] = torch.from_numpy(idx).to(dev)
+    y = pipe.step(dev_inp)
+    assert int(y.view(torch.int16).abs().max()) == 0
+    assert pipe.buf.check() == 0
+
+
+def test_mask_rank0_decode(dev):
+    """DeepEP issue #84 masking: every pick of rank 0's experts set to -1; rank 0
+    then receives nothing and combine ignores the masked picks."""
+    w = wl.get("decode")
+    inp = wl.generate(w)
+    idx = inp["topk_idx"].copy()
+    idx[idx // w.L == 0] = -1
+    inp["topk_idx"] = idx
+    pipe, *_ = full_check(w.with_(name="decode_masked"), dev, inp=inp)
+    rc = pipe.buf.recv_count.cpu().numpy().reshape(w.P, w.L, w.P)
+    assert rc[0].sum() == 0
+
+
+def test_repeated_calls_are_identical(dev):
+    """The layout's ticket counter re-arms itself; a second pass over the same
+    inputs reproduces every output bit for bit and raises no error bits."""
+    w = wl.get("skewed")
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev)
+    outs = []
+    for _ in range(3):
+        pipe.layout(dev_inp)
+        pipe.dispatch(dev_inp)
+        torch.cuda.synchronize()
+        outs.append([t.clone() for t in (pipe.buf.expert_count, pipe.buf.expert_offset,
+                                         pipe.buf.recv_count, pipe.buf.dst_pos,
+                                         pipe.buf.token_scale)])
+    for a, b in zip(outs[0], outs[-1]):
+        assert torch.equal(a, b)
+    assert pipe.buf.check() == 0
+
+
+def test_roundtrip_identity_decode_shape_bf16(dev):
+    """combine(dispatch(x)) == x with one-hot weights at the decode shape in bf16."""
+    w = wl.get("decode").with_(name="decode_q0", quant_mode=0)
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev, alias_expert_out=True)
+    rng = np.random.default_rng(2)
+    onehot = np.zeros((w.B, w.k), np.float32)
+    onehot[np.arange(w.B), rng.integers(0, w.k, w.B)] = 1.0
+    dev_inp["topk_weights"] = torch.from_numpy(onehot).to(dev)
+    y = pipe.step(dev_inp)
+    assert torch.equal(y.view(torch.int16), dev_inp["x"].view(torch.int16))
