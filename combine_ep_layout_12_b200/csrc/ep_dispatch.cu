@@ -198,10 +198,10 @@ __global__ void __launch_bounds__(256) dispatch_bf16_kernel(DispatchArgs a) {
     }
 }
 
-int pick_units(int n, int* U, int* NT) {
-    // smallest U in {1,2,4,8} with ceil(n / U) <= 256 threads
+int pick_units(int n, int max_u, int* U, int* NT) {
+    // smallest power-of-two U <= max_u with ceil(n / U) <= 256 threads
     int u = 1;
-    while (u < 8 && (n + u - 1) / u > 256) u *= 2;
+    while (u < max_u && (n + u - 1) / u > 256) u *= 2;
     int nt = (n + u - 1) / u;
     nt = ((nt + 31) / 32) * 32;
     if (nt > 256) return EP_ERR_UNSUPPORTED;
@@ -230,7 +230,7 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
     cudaError_t e = cudaSuccess;
     const dim3 grid(s.B);
     if (s.quant_mode == 2) {
-        if (pick_units(s.d / 16, &U, &NT) != EP_OK) return EP_ERR_UNSUPPORTED;
+        if (pick_units(s.d / 16, 8, &U, &NT) != EP_OK) return EP_ERR_UNSUPPORTED;
         switch (U) {
             case 1: e = launch_pdl(dispatch_int8_kernel<1>, grid, dim3(NT), 0, stream, a); break;
             case 2: e = launch_pdl(dispatch_int8_kernel<2>, grid, dim3(NT), 0, stream, a); break;
@@ -238,14 +238,13 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
             default: e = launch_pdl(dispatch_int8_kernel<8>, grid, dim3(NT), 0, stream, a); break;
         }
     } else {
-        if (pick_units(s.d / 8, &U, &NT) != EP_OK) {
-            return EP_ERR_UNSUPPORTED;
-        }
+        if (pick_units(s.d / 8, 16, &U, &NT) != EP_OK) return EP_ERR_UNSUPPORTED;
         switch (U) {
             case 1: e = launch_pdl(dispatch_bf16_kernel<1>, grid, dim3(NT), 0, stream, a); break;
             case 2: e = launch_pdl(dispatch_bf16_kernel<2>, grid, dim3(NT), 0, stream, a); break;
             case 4: e = launch_pdl(dispatch_bf16_kernel<4>, grid, dim3(NT), 0, stream, a); break;
-            default: e = launch_pdl(dispatch_bf16_kernel<8>, grid, dim3(NT), 0, stream, a); break;
+            case 8: e = launch_pdl(dispatch_bf16_kernel<8>, grid, dim3(NT), 0, stream, a); break;
+            default: e = launch_pdl(dispatch_bf16_kernel<16>, grid, dim3(NT), 0, stream, a); break;
         }
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;

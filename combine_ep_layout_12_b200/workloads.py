@@ -72,6 +72,10 @@ WORKLOADS = {
                         smooth="ones"),
     # DeepSeek-V3-shaped low-latency decode: 8 ranks x 128 tokens, 256 experts, top-8, int8
     "decode": Workload("decode", B=1024, d=7168, k=8, P=8, M=128, E=256, quant_mode=2),
+    # the decode kernels on a smaller receive buffer (64 experts: 1.4 GB instead of
+    # 5.6 GB of device buffers; same B, d, k and routed rows per launch), used for
+    # multi-pass profiler captures
+    "decode_e64": Workload("decode_e64", B=1024, d=7168, k=8, P=8, M=128, E=64, quant_mode=2),
     # high-throughput prefill: 8 ranks x 4096 tokens, bf16 payload
     "prefill": Workload("prefill", B=32768, d=7168, k=8, P=8, M=4096, E=256, quant_mode=0),
     # skewed Zipf(1.2) routing over 64 routed + 1 zero + 1 copy + 1 const experts, top-6
