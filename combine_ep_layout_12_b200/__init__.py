@@ -12,12 +12,12 @@ import torch
 
 from . import _binding as abi
 from ._binding import (EPError, ep_buffer_check, ep_buffer_create, ep_buffer_destroy,
-                       ep_buffer_size, ep_combine, ep_dispatch, ep_layout, ep_status_str,
-                       make_config)
+                       ep_buffer_size, ep_combine, ep_dispatch, ep_layout,
+                       ep_layout_static_scratch, ep_status_str, make_config)
 
 __all__ = ["EPBuffer", "EPError", "abi", "ep_buffer_check", "ep_buffer_create",
            "ep_buffer_destroy", "ep_buffer_size", "ep_combine", "ep_dispatch", "ep_layout",
-           "ep_status_str", "make_config"]
+           "ep_layout_static_scratch", "ep_status_str", "make_config"]
 
 
 def _ptr(t):

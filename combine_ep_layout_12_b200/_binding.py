@@ -65,8 +65,9 @@ def lib():
     L.ep_dispatch.argtypes = [vp, vp, vp, vp]
     L.ep_combine.argtypes = [vp] * 10
     L.ep_buffer_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.ep_layout_static_scratch.argtypes = [ctypes.POINTER(ep_config)] + [vp] * 8
     for f in (L.ep_buffer_size, L.ep_buffer_create, L.ep_buffer_destroy, L.ep_layout,
-              L.ep_dispatch, L.ep_combine, L.ep_buffer_check):
+              L.ep_dispatch, L.ep_combine, L.ep_buffer_check, L.ep_layout_static_scratch):
         f.restype = i
     L.ep_status_str.argtypes = [i]
     L.ep_status_str.restype = ctypes.c_char_p
@@ -122,3 +123,13 @@ def ep_buffer_check(handle, stream=0):
     bits = ctypes.c_uint32()
     _check(lib().ep_buffer_check(handle, stream, ctypes.byref(bits)), "ep_buffer_check")
     return int(bits.value)
+
+
+def ep_layout_static_scratch(cfg, topk_idx, expert_count, expert_offset, recv_count, dst_pos,
+                             recv_src, err_word=None, stream=0):
+    """Layout without a caller workspace (scratch in the library's static device
+    memory); for callers that cannot allocate.  All arguments after cfg are device
+    addresses (ints); err_word may be None."""
+    _check(lib().ep_layout_static_scratch(ctypes.byref(cfg), topk_idx, expert_count,
+                                          expert_offset, recv_count, dst_pos, recv_src,
+                                          err_word, stream), "ep_layout_static_scratch")

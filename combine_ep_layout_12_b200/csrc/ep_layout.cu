@@ -18,6 +18,8 @@
 // i.e. its rank among rank r's tokens that routed to g, in ascending token order.
 // The last CTA to finish (a ticket counter in the workspace; no CTA ever waits on
 // another) adds the per-rank counts into expert_count and scans expert_offset.
+#include <mutex>
+
 #include "ep_internal.cuh"
 
 namespace ep {
@@ -241,4 +243,84 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// ep_layout_static_scratch: the layout for callers that cannot allocate.
+//
+// The regular entry point keeps its scratch (ticket counter, error word, per-rank
+// special-expert counts) in a workspace the caller allocates.  Some callers have
+// no way to do that: a serving engine that has already handed every byte of the
+// GPU to its own pool, code that must not call cudaMalloc because it can
+// synchronize the whole device and stall other streams, or a plain C host without
+// a tensor library.  This variant keeps that scratch in a fixed array in the
+// library's own device memory instead.  It launches the same layout kernel.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = 64 * 1024;  // 256-byte header + P*(Z+C+K) int32 counts
+
+// Lives on every GPU that loads this library, until the process exits.
+static __device__ __align__(256) unsigned char g_layout_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+// Device address of g_layout_scratch on the current device.  Looked up once per
+// device with that device current; in host code the symbol itself is only a
+// host-side stand-in and must never be handed to a kernel.
+cudaError_t static_scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_layout_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
 }  // namespace ep
+
+extern "C" int ep_layout_static_scratch(const ep_config* cfg, const int32_t* topk_idx,
+                                        int32_t* expert_count, int32_t* expert_offset,
+                                        int32_t* recv_count, int32_t* dst_pos, int32_t* recv_src,
+                                        uint32_t* err_word, ep_stream_t stream) {
+    ep_buffer_sizes sz;
+    const int st = ep_buffer_size(cfg, &sz);  // validates cfg
+    if (st != EP_OK) return st;
+    if (sz.workspace > ep::kStaticScratchBytes) return EP_ERR_CAPACITY;
+    auto bad = [](const void* p, size_t size) {
+        return size != 0 && (p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) != 0);
+    };
+    if (bad(expert_count, sz.expert_count) || bad(expert_offset, sz.expert_offset) ||
+        bad(recv_count, sz.recv_count) || bad(dst_pos, sz.dst_pos) || bad(recv_src, sz.recv_src) ||
+        bad(topk_idx, sz.dst_pos) || bad(err_word, err_word ? 4 : 0))
+        return EP_ERR_INVALID_ARG;
+    void* scratch = nullptr;
+    if (ep::static_scratch_address(&scratch) != cudaSuccess) return EP_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // The array keeps the previous call's contents: start from zero every call.
+    if (cudaMemsetAsync(scratch, 0, sz.workspace, s) != cudaSuccess) return EP_ERR_CUDA;
+    ep_buffer_ptrs p = {};
+    p.expert_count = expert_count;
+    p.expert_offset = expert_offset;
+    p.recv_count = recv_count;
+    p.dst_pos = dst_pos;
+    p.recv_src = recv_src;
+    p.workspace = scratch;
+    const int lst = ep::launch_layout(ep::make_shape(*cfg), p, topk_idx, s);
+    if (lst != EP_OK) return lst;
+    if (err_word) {
+        const auto* hdr = reinterpret_cast<const ep::WsHeader*>(scratch);
+        if (cudaMemcpyAsync(err_word, &hdr->err, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+            return EP_ERR_CUDA;
+    }
+    return EP_OK;
+}

@@ -173,6 +173,36 @@ EP_API int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t*
                const float* topk_weights, const uint16_t* ori_x, const uint16_t* a1,
                const uint16_t* a2, const uint16_t* v, uint16_t* y, ep_stream_t stream);
 
+/* Layout for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this entry point; it exists for this library's users.
+ *
+ * Same outputs, bit for bit, as ep_layout on the same topk_idx, but without an
+ * ep_buffer or a workspace: the caller passes only the inputs and the outputs
+ * (device arrays sized as ep_buffer_size reports; cfg is validated the same
+ * way).  Meant for callers that cannot allocate a workspace: an engine whose
+ * memory pool already owns all of the GPU's memory, code that must not call
+ * cudaMalloc because it can synchronize the device and stall other streams, or
+ * a plain C host without a tensor library.  This call itself allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library routine).
+ *
+ * Its scratch is a 64 KiB array in the library's static device memory, present
+ * on every GPU that loads the library until the process exits.  It holds a
+ * 256-byte header plus one int32 per (rank, special expert), so configurations
+ * with P * (Z + C + K) > 16320 are rejected with EP_ERR_CAPACITY.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array, and each call clears the part
+ *    it uses on `stream` first.  Calls whose work can overlap on the GPU (other
+ *    streams, other host threads) race on it: order them on one stream.
+ *  - err_word: device uint32 that receives this call's error bits (EP_ERRBIT_*,
+ *    overwritten, not OR-ed); NULL to not report them.
+ * Returns EP_OK, a validation status, EP_ERR_CAPACITY or EP_ERR_CUDA. */
+EP_API int ep_layout_static_scratch(const ep_config* cfg, const int32_t* topk_idx,
+                                    int32_t* expert_count, int32_t* expert_offset,
+                                    int32_t* recv_count, int32_t* dst_pos, int32_t* recv_src,
+                                    uint32_t* err_word, ep_stream_t stream);
+
 /* Synchronize `stream`, read the device error word into *err_bits and clear it. */
 EP_API int ep_buffer_check(ep_buffer* buf, ep_stream_t stream, uint32_t* err_bits);
 
