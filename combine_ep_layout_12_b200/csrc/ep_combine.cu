@@ -49,15 +49,18 @@ __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
 }
 
 template <int KMAX>
-__global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(CombineArgs a) {
     __shared__ int s_kind[KMAX];
     __shared__ long long s_src[KMAX];  // receive row (routed) or const index
     __shared__ float s_w[KMAX];
 
+    // CTA = (token t, column slice c); the slice is swept by the CTA's threads
     const int t = blockIdx.x / a.chunks;
-    const int chunk = blockIdx.x - t * a.chunks;
+    const int c = blockIdx.x - t * a.chunks;
     const int nvec = a.d >> 3;
-    const int vcol = chunk * blockDim.x + threadIdx.x;
+    const int span = (nvec + a.chunks - 1) / a.chunks;
+    const int v_begin = c * span;
+    const int v_end = min(nvec, v_begin + span);
 
     pdl_wait();
     pdl_launch_dependents();
@@ -88,50 +91,52 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
     }
     if (threadIdx.x < 32) report_err(a.err, bad);
     __syncthreads();
-    if (vcol >= nvec) return;
 
-    const size_t col = (size_t)vcol * 8;
-    uint4 raw[KMAX];
+    for (int vcol = v_begin + threadIdx.x; vcol < v_end; vcol += blockDim.x) {
+        const size_t col = (size_t)vcol * 8;
+        uint4 raw[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        raw[j] = make_uint4(0, 0, 0, 0);
-        if (j < a.k) {
+        for (int j = 0; j < KMAX; ++j) {
+            raw[j] = make_uint4(0, 0, 0, 0);
+            if (j < a.k) {
+                const int kind = s_kind[j];
+                if (kind == kRouted)
+                    raw[j] = ld_stream_v4(a.expert_out + (size_t)s_src[j] * a.d + col);
+                else if (kind != kSkip)
+                    raw[j] = ld_stream_v4(a.ori_x + (size_t)t * a.d + col);
+            }
+        }
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KMAX; ++j) {
+            if (j >= a.k) continue;
             const int kind = s_kind[j];
-            if (kind == kRouted)
-                raw[j] = ld_stream_v4(a.expert_out + (size_t)s_src[j] * a.d + col);
-            else if (kind != kSkip)
-                raw[j] = ld_stream_v4(a.ori_x + (size_t)t * a.d + col);
+            if (kind == kSkip) continue;
+            float e[8];
+            unpack8(raw[j], e);
+            if (kind == kConst) {
+                const size_t off = (size_t)s_src[j] * a.d + col;
+                float f1[8], f2[8], fv[8];
+                unpack8(ld_stream_v4(a.a1 + off), f1);
+                unpack8(ld_stream_v4(a.a2 + off), f2);
+                unpack8(ld_stream_v4(a.v + off), fv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    e[i] = __fadd_rn(__fmul_rn(f1[i], e[i]), __fmul_rn(f2[i], fv[i]));
+            }
+            const float w = s_w[j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(w, e[i], acc[i]);
         }
+        uint4 out;
+        out.x = pack_bf16x2(acc[0], acc[1]);
+        out.y = pack_bf16x2(acc[2], acc[3]);
+        out.z = pack_bf16x2(acc[4], acc[5]);
+        out.w = pack_bf16x2(acc[6], acc[7]);
+        st_v4(a.y + (size_t)t * a.d + col, out);
     }
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-        if (j >= a.k) continue;
-        const int kind = s_kind[j];
-        if (kind == kSkip) continue;
-        float e[8];
-        unpack8(raw[j], e);
-        if (kind == kConst) {
-            const size_t off = (size_t)s_src[j] * a.d + col;
-            float f1[8], f2[8], fv[8];
-            unpack8(ld_stream_v4(a.a1 + off), f1);
-            unpack8(ld_stream_v4(a.a2 + off), f2);
-            unpack8(ld_stream_v4(a.v + off), fv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) e[i] = __fadd_rn(__fmul_rn(f1[i], e[i]), __fmul_rn(f2[i], fv[i]));
-        }
-        const float w = s_w[j];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(w, e[i], acc[i]);
-    }
-    uint4 out;
-    out.x = pack_bf16x2(acc[0], acc[1]);
-    out.y = pack_bf16x2(acc[2], acc[3]);
-    out.z = pack_bf16x2(acc[4], acc[5]);
-    out.w = pack_bf16x2(acc[6], acc[7]);
-    st_v4(a.y + (size_t)t * a.d + col, out);
 }
 
 }  // namespace
@@ -159,9 +164,16 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
     a.Z = s.Z;
     a.C = s.C;
     a.K = s.K;
+    // One CTA per token when that fills the GPU in about one wave; otherwise split
+    // each token's columns over up to nvec / NT CTAs.
     const int nvec = s.d / 8;
-    int NT = nvec < 128 ? ((nvec + 31) / 32) * 32 : 128;
-    a.chunks = (nvec + NT - 1) / NT;
+    const int NT = nvec < 128 ? ((nvec + 31) / 32) * 32 : 128;
+    const int max_chunks = (nvec + NT - 1) / NT;
+    const long long target = (long long)num_sms() * 7;
+    long long chunks = target / (s.B > 0 ? s.B : 1);
+    if (chunks < 1) chunks = 1;
+    if (chunks > max_chunks) chunks = max_chunks;
+    a.chunks = (int)chunks;
     const long long nblocks = (long long)s.B * a.chunks;
     if (nblocks > 0x7fffffffLL) return EP_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)nblocks);

@@ -14,6 +14,7 @@ struct ep_buffer {
     ep_config cfg;
     ep_buffer_ptrs ptrs;
     ep_buffer_sizes sizes;
+    const int32_t* last_topk_idx;  // routing of the latest ep_layout (dispatch may re-read it)
 };
 
 namespace {
@@ -94,6 +95,7 @@ int ep_buffer_create(const ep_config* cfg, const ep_buffer_ptrs* ptrs, ep_buffer
     b->cfg = *cfg;
     b->ptrs = *ptrs;
     b->sizes = s;
+    b->last_topk_idx = nullptr;
     *out = b;
     return EP_OK;
 }
@@ -106,8 +108,10 @@ int ep_buffer_destroy(ep_buffer* buf) {
 int ep_layout(ep_buffer* buf, const int32_t* topk_idx, ep_stream_t stream) {
     if (!buf) return EP_ERR_INVALID_ARG;
     if (buf->cfg.B > 0 && (!topk_idx || !aligned4(topk_idx))) return EP_ERR_INVALID_ARG;
-    return ep::launch_layout(ep::make_shape(buf->cfg), buf->ptrs, topk_idx,
-                             reinterpret_cast<cudaStream_t>(stream));
+    const int st = ep::launch_layout(ep::make_shape(buf->cfg), buf->ptrs, topk_idx,
+                                     reinterpret_cast<cudaStream_t>(stream));
+    buf->last_topk_idx = st == EP_OK ? topk_idx : nullptr;
+    return st;
 }
 
 int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale, ep_stream_t stream) {
@@ -116,7 +120,7 @@ int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale, ep
     if (c.B > 0 && (!x || !aligned16(x))) return EP_ERR_INVALID_ARG;
     if (smooth_scale && (c.smooth_rows == 0 || !aligned16(smooth_scale))) return EP_ERR_INVALID_ARG;
     if (smooth_scale && c.quant_mode != 2) return EP_ERR_INVALID_ARG;
-    return ep::launch_dispatch(ep::make_shape(c), buf->ptrs, x, smooth_scale,
+    return ep::launch_dispatch(ep::make_shape(c), buf->ptrs, x, smooth_scale, buf->last_topk_idx,
                                reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -45,12 +45,28 @@ inline Shape make_shape(const ep_config& c) {
 // Host launchers (one per kernel family); each returns an EP_* status.
 int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
                   cudaStream_t stream);
+// topk_idx: the routing of the latest layout on this buffer (lets dispatch derive
+// its receive rows itself for small per-rank batches); may be null.
 int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
-                    const float* smooth, cudaStream_t stream);
+                    const float* smooth, const int32_t* topk_idx, cudaStream_t stream);
 int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
                    const int32_t* topk_idx, const float* topk_weights, const uint16_t* ori_x,
                    const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
                    cudaStream_t stream);
+
+// Streaming multiprocessors of the current device (queried once per device).
+inline int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
 
 // Launch with programmatic dependent launch enabled: the kernel may begin while
 // the previous kernel on the stream drains; every kernel here executes

@@ -38,6 +38,222 @@ struct LayoutArgs {
     int warps;            // warps per CTA
 };
 
+// Exclusive prefix of cnt[0..n) into out[0..n], out[n] = total; all threads of the
+// CTA call it.  Thread i owns a contiguous chunk; chunk sums go through a warp
+// shuffle scan and one pass over the warp totals.  wsum: 32 ints of shared memory.
+__device__ void block_exclusive_scan(const int* cnt, int n, int32_t* out, int* wsum) {
+    const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int lo = min(n, (int)threadIdx.x * per);
+    const int hi = min(n, lo + per);
+    int local = 0;
+    for (int g = lo; g < hi; ++g) local += cnt[g];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = (blockDim.x + 31) >> 5;
+        int v = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += y;
+        }
+        wsum[lane] = v;
+    }
+    __syncthreads();
+    int acc = x - local + (warp > 0 ? wsum[warp - 1] : 0);
+    for (int g = lo; g < hi; ++g) {
+        out[g] = acc;
+        acc += cnt[g];
+    }
+    if (threadIdx.x == blockDim.x - 1) out[n] = acc;
+}
+
+// Pick ids of token t into ids[0..k), -1 beyond k.  16-byte loads when each row
+// starts on a 16-byte boundary (k % 4 == 0 and an aligned base).
+template <int KM>
+__device__ __forceinline__ void load_token_ids(const int32_t* topk_idx, int t, int k, bool vec4,
+                                               int* ids) {
+    if (vec4) {
+        const int4* src = reinterpret_cast<const int4*>(topk_idx + (size_t)t * k);
+#pragma unroll
+        for (int j4 = 0; j4 < KM / 4; ++j4) {
+            int4 v = make_int4(-1, -1, -1, -1);
+            if (4 * j4 < k) v = __ldg(src + j4);
+            ids[4 * j4] = v.x;
+            ids[4 * j4 + 1] = v.y;
+            ids[4 * j4 + 2] = v.z;
+            ids[4 * j4 + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < KM; ++j) ids[j] = (j < k) ? __ldg(topk_idx + (size_t)t * k + j) : -1;
+    }
+}
+
+// Classify the picks of one token: returns a mask with bit j set when pick j is
+// routed (the first occurrence of an id in [0, E)); repeated routed ids and ids
+// outside [-1, E_tot) set error bits; specials are handed to on_special.
+template <int KM, typename OnSpecial>
+__device__ __forceinline__ unsigned classify_ids(const int* ids, int k, int E, int E_tot,
+                                                 unsigned& err, OnSpecial on_special) {
+    unsigned routed = 0;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        if (j >= k) continue;
+        const int g = ids[j];
+        if (g == -1) continue;
+        if (g < -1 || g >= E_tot) {
+            err |= EP_ERRBIT_BAD_ID;
+            continue;
+        }
+        if (g >= E) {
+            on_special(g - E);
+            continue;
+        }
+        bool dup = false;
+#pragma unroll
+        for (int jj = 0; jj < KM; ++jj)
+            if (jj < j && ids[jj] == g) dup = true;
+        if (dup) {
+            err |= EP_ERRBIT_DUP_ID;
+            continue;
+        }
+        routed |= 1u << j;
+    }
+    return routed;
+}
+
+// Layout for small per-rank batches (T <= 256), with no dependency between CTAs.
+//  - CTA 0 (the count CTA) histograms every token's routed ids per (expert, rank)
+//    and the special ids, and writes recv_count, expert_count and expert_offset.
+//  - Every other CTA holds 8 warps; warp q handles the q-th 32-token chunk of a
+//    rank.  It counts, per expert, the rank's tokens before its chunk (read from
+//    L2; a token counts once per expert), sets one lane bit per routed id of its
+//    own tokens, and a token's slot is  before[g] + popc(mask[g] & lanemask_lt),
+//    i.e. its rank among the rank's tokens that routed to g, in token order.
+// Both halves only use order-independent shared-memory atomics, so the result is
+// deterministic.
+template <int KM>
+__global__ void __launch_bounds__(256) layout_small_kernel(LayoutArgs a, int cpr) {
+    extern __shared__ unsigned smem[];
+    const int E = a.E, k = a.k, P = a.P;
+    const bool vec4 = (k % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.topk_idx) & 15) == 0);
+    unsigned err = 0;
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    if (blockIdx.x == 0) {
+        int* cnt = reinterpret_cast<int*>(smem);     // [E][P]
+        int* spc = cnt + (size_t)E * P;               // [n_special]
+        int* ec = spc + a.n_special;                  // [E_tot]
+        int* wsum = ec + a.E_tot;                     // [32]
+        for (int i = threadIdx.x; i < E * P; i += blockDim.x) cnt[i] = 0;
+        for (int i = threadIdx.x; i < a.n_special; i += blockDim.x) spc[i] = 0;
+        __syncthreads();
+        // four tokens per thread per pass, their id loads issued together
+        const int stride = blockDim.x;
+        for (int t0 = threadIdx.x; t0 < a.B; t0 += 4 * stride) {
+            int ids[4][KM];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int t = t0 + b * stride;
+                if (t < a.B) {
+                    load_token_ids<KM>(a.topk_idx, t, k, vec4, ids[b]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < KM; ++j) ids[b][j] = -1;
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int t = t0 + b * stride;
+                if (t >= a.B) continue;
+                const int r = t / a.T;
+                const unsigned rb = classify_ids<KM>(ids[b], k, E, a.E_tot, err,
+                                                 [&](int sidx) { atomicAdd(&spc[sidx], 1); });
+#pragma unroll
+                for (int j = 0; j < KM; ++j)
+                    if (rb & (1u << j)) atomicAdd(&cnt[(size_t)ids[b][j] * P + r], 1);
+            }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < E * P; i += blockDim.x) a.recv_count[i] = cnt[i];
+        for (int gg = threadIdx.x; gg < a.E_tot; gg += blockDim.x) {
+            int v = 0;
+            if (gg < E) {
+                for (int rr = 0; rr < P; ++rr) v += cnt[(size_t)gg * P + rr];
+            } else {
+                v = spc[gg - E];
+            }
+            ec[gg] = v;
+            a.expert_count[gg] = v;
+        }
+        report_err(&a.ws->err, err);
+        __syncthreads();
+        block_exclusive_scan(ec, a.E_tot, a.expert_offset, wsum);
+        return;
+    }
+
+    // slot CTAs
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = (blockIdx.x - 1) * (blockDim.x >> 5) + warp;  // chunk id
+    if (q >= P * cpr) return;  // no barrier below: whole warps leave together
+    const int r = q / cpr, c = q - r * cpr;
+    int* before = reinterpret_cast<int*>(smem) + (size_t)warp * E * 2;  // [E]
+    unsigned* mask = reinterpret_cast<unsigned*>(before + E);          // [E]
+    for (int g = lane; g < E; g += 32) {
+        before[g] = 0;
+        mask[g] = 0u;
+    }
+    __syncwarp();
+    unsigned ignore = 0;
+    for (int t = a.T * r + lane; t < a.T * r + c * 32; t += 32) {
+        int ids[KM];
+        load_token_ids<KM>(a.topk_idx, t, k, vec4, ids);
+        const unsigned rb = classify_ids<KM>(ids, k, E, a.E_tot, ignore, [](int) {});
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            if (rb & (1u << j)) atomicAdd(&before[ids[j]], 1);
+    }
+    const int t = a.T * r + c * 32 + lane;
+    const bool valid = c * 32 + lane < a.T;
+    int ids[KM];
+    unsigned rb = 0;
+    if (valid) {
+        load_token_ids<KM>(a.topk_idx, t, k, vec4, ids);
+        rb = classify_ids<KM>(ids, k, E, a.E_tot, err, [](int) {});
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+        if (rb & (1u << j)) atomicOr(&mask[ids[j]], 1u << lane);
+    __syncwarp();
+    if (valid) {
+        const unsigned lt = lanemask_lt();
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            if (j >= k) continue;
+            int row = -1;
+            if (rb & (1u << j)) {
+                const int g = ids[j];
+                row = g * P * a.M + r * a.M + before[g] + __popc(mask[g] & lt);
+                a.recv_src[row] = t;
+            }
+            a.dst_pos[(size_t)t * k + j] = row;
+        }
+    }
+    // errors of the chunk's own tokens only (the count CTA reports the same bits)
+    report_err(&a.ws->err, err);
+}
+
+template <int KM>
 __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
     extern __shared__ unsigned smem[];
     const int W = a.warps;
@@ -74,17 +290,17 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
 
         const int t = round0 + warp * 32 + lane;
         const bool valid = t < tok_end;
-        int ids[kMaxK];
-        bool routed[kMaxK];
+        int ids[KM];
+        bool routed[KM];
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
+        for (int j = 0; j < KM; ++j) {
             ids[j] = -1;
             routed[j] = false;
             if (j < k && valid) ids[j] = a.topk_idx[(size_t)t * k + j];
         }
         // (2) classify; routed ids set their lane bit
 #pragma unroll
-        for (int j = 0; j < kMaxK; ++j) {
+        for (int j = 0; j < KM; ++j) {
             if (j >= k || !valid) continue;
             const int g = ids[j];
             if (g == -1) continue;
@@ -98,7 +314,7 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
             }
             bool dup = false;
 #pragma unroll
-            for (int jj = 0; jj < kMaxK; ++jj)
+            for (int jj = 0; jj < KM; ++jj)
                 if (jj < j && ids[jj] == g) dup = true;
             if (dup) {
                 err |= EP_ERRBIT_DUP_ID;
@@ -123,7 +339,7 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
         if (valid) {
             const unsigned lt = lanemask_lt();
 #pragma unroll
-            for (int j = 0; j < kMaxK; ++j) {
+            for (int j = 0; j < KM; ++j) {
                 if (j >= k) continue;
                 int row = -1;
                 if (routed[j]) {
@@ -155,43 +371,26 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
     if (!s_last) return;
     __threadfence();
 
-    // expert_count over all ids, then exclusive prefix into expert_offset.
-    // Thread i owns a contiguous chunk of ids; chunk sums are scanned in smem.
-    int* chunk = reinterpret_cast<int*>(smem);  // reuse: [blockDim]
-    const int n = a.E_tot;
-    const int per = (n + blockDim.x - 1) / blockDim.x;
-    const int lo = min(n, (int)threadIdx.x * per);
-    const int hi = min(n, lo + per);
-    int sum = 0;
-    for (int g = lo; g < hi; ++g) {
-        int c = 0;
+    // expert_count over all ids, then its exclusive prefix into expert_offset.
+    // The rank loop is unrolled so a thread's loads are in flight together.
+    int* ec = reinterpret_cast<int*>(smem);            // reuse: [E_tot]
+    int* wsum = ec + a.E_tot;                          // [32]
+    for (int g = threadIdx.x; g < a.E_tot; g += blockDim.x) {
+        int v = 0;
         if (g < E) {
-            for (int q = 0; q < a.P; ++q) c += __ldcg(&a.recv_count[(size_t)g * a.P + q]);
+            const int32_t* src = a.recv_count + (size_t)g * a.P;
+#pragma unroll 8
+            for (int q = 0; q < a.P; ++q) v += __ldcg(src + q);
         } else {
-            for (int q = 0; q < a.P; ++q)
-                c += __ldcg(&a.sp_partial[(size_t)q * a.n_special + (g - E)]);
+#pragma unroll 8
+            for (int q = 0; q < a.P; ++q) v += __ldcg(&a.sp_partial[(size_t)q * a.n_special + (g - E)]);
         }
-        a.expert_count[g] = c;
-        sum += c;
-    }
-    chunk[threadIdx.x] = sum;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int i = 0; i < (int)blockDim.x; ++i) {
-            const int v = chunk[i];
-            chunk[i] = acc;
-            acc += v;
-        }
-        a.expert_offset[n] = acc;
-        a.ws->done = 0u;  // re-arm the ticket for the next launch
+        ec[g] = v;
+        a.expert_count[g] = v;
     }
     __syncthreads();
-    int acc = chunk[threadIdx.x];
-    for (int g = lo; g < hi; ++g) {
-        a.expert_offset[g] = acc;
-        acc += __ldcg(&a.expert_count[g]);
-    }
+    block_exclusive_scan(ec, a.E_tot, a.expert_offset, wsum);
+    if (threadIdx.x == 0) a.ws->done = 0u;  // re-arm the ticket for the next launch
 }
 
 }  // namespace
@@ -205,24 +404,70 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         cudaError_t e3 = cudaMemsetAsync(p.recv_count, 0, sizeof(int32_t) * s.E * s.P, stream);
         return (e1 || e2 || e3) ? EP_ERR_CUDA : EP_OK;
     }
-    // warps per CTA: enough for one round of the rank's tokens, at most 32,
-    // within the shared-memory budget (two [warps][E] arrays plus [E] + specials)
     const size_t budget = 160 * 1024;
+    static bool attr_small[16] = {false};
+    int dev0 = 0;
+    cudaGetDevice(&dev0);
+    // small per-rank batches: count CTA + slot CTAs, no inter-CTA dependency
+    const int cpr = (s.T + 31) / 32;
+    const size_t smem_count = sizeof(int) * ((size_t)s.E * s.P + s.n_special + s.E_tot + 32);
+    const size_t smem_slot = sizeof(int) * (size_t)8 * s.E * 2;
+    const size_t smem_small = smem_count > smem_slot ? smem_count : smem_slot;
+    if (s.T <= 256 && smem_small <= budget) {
+        if (dev0 < 16 && !attr_small[dev0]) {
+            if (cudaFuncSetAttribute(layout_small_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+                cudaFuncSetAttribute(layout_small_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+                cudaFuncSetAttribute(layout_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+                cudaFuncSetAttribute(layout_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget))
+                return EP_ERR_CUDA;
+            attr_small[dev0] = true;
+        }
+        LayoutArgs a1;
+        a1.topk_idx = topk_idx;
+        a1.expert_count = p.expert_count;
+        a1.expert_offset = p.expert_offset;
+        a1.recv_count = p.recv_count;
+        a1.dst_pos = p.dst_pos;
+        a1.recv_src = p.recv_src;
+        a1.ws = reinterpret_cast<WsHeader*>(p.workspace);
+        a1.sp_partial = nullptr;
+        a1.B = s.B; a1.k = s.k; a1.P = s.P; a1.M = s.M; a1.E = s.E; a1.T = s.T;
+        a1.n_special = s.n_special; a1.E_tot = s.E_tot;
+        a1.warps = 8;
+        const int nchunks = s.P * cpr;
+        const int grid = 1 + (nchunks + 7) / 8;
+        cudaError_t e;
+        if (s.k <= 2)
+            e = launch_pdl(layout_small_kernel<2>, dim3(grid), dim3(256), smem_small, stream, a1, cpr);
+        else if (s.k <= 4)
+            e = launch_pdl(layout_small_kernel<4>, dim3(grid), dim3(256), smem_small, stream, a1, cpr);
+        else if (s.k <= 8)
+            e = launch_pdl(layout_small_kernel<8>, dim3(grid), dim3(256), smem_small, stream, a1, cpr);
+        else
+            e = launch_pdl(layout_small_kernel<16>, dim3(grid), dim3(256), smem_small, stream, a1, cpr);
+        return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    }
+    // multi-CTA path: one CTA per rank; warps per CTA enough for one round of the
+    // rank's tokens, at most 32, within the shared-memory budget (two [warps][E]
+    // arrays plus [E] + specials)
     const size_t fixed = sizeof(int) * ((size_t)s.E + s.n_special);
     int warps = (s.T + 31) / 32;
     if (warps > 32) warps = 32;
     if (warps < 1) warps = 1;
     while (warps > 1 && fixed + (size_t)warps * s.E * 8 > budget) --warps;
     size_t smem = fixed + (size_t)warps * s.E * 8;
-    const size_t need_tail = sizeof(int) * (size_t)warps * 32;  // chunk sums of the last CTA
+    const size_t need_tail = sizeof(int) * ((size_t)s.E_tot + 32);  // counts + scan of the last CTA
     if (smem < need_tail) smem = need_tail;
+    if (smem > budget) return EP_ERR_UNSUPPORTED;
 
     static bool attr_set[16] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 16 && !attr_set[dev]) {
-        if (cudaFuncSetAttribute(layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)budget) != cudaSuccess)
+        if (cudaFuncSetAttribute(layout_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+            cudaFuncSetAttribute(layout_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+            cudaFuncSetAttribute(layout_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+            cudaFuncSetAttribute(layout_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget))
             return EP_ERR_CUDA;
         attr_set[dev] = true;
     }
@@ -239,7 +484,15 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     a.B = s.B; a.k = s.k; a.P = s.P; a.M = s.M; a.E = s.E; a.T = s.T;
     a.n_special = s.n_special; a.E_tot = s.E_tot;
     a.warps = warps;
-    cudaError_t e = launch_pdl(layout_kernel, dim3(s.P), dim3(warps * 32), smem, stream, a);
+    cudaError_t e;
+    if (s.k <= 2)
+        e = launch_pdl(layout_kernel<2>, dim3(s.P), dim3(warps * 32), smem, stream, a);
+    else if (s.k <= 4)
+        e = launch_pdl(layout_kernel<4>, dim3(s.P), dim3(warps * 32), smem, stream, a);
+    else if (s.k <= 8)
+        e = launch_pdl(layout_kernel<8>, dim3(s.P), dim3(warps * 32), smem, stream, a);
+    else
+        e = launch_pdl(layout_kernel<16>, dim3(s.P), dim3(warps * 32), smem, stream, a);
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 

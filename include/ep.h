@@ -157,9 +157,13 @@ EP_API int ep_buffer_destroy(ep_buffer* buf);
 EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, ep_stream_t stream);
 
 /* Quantize (quant_mode 2) or pass through (0) x (bf16 [B][d], device) and scatter
- * every routed pick into recv_x (plus recv_scale, token_scale in mode 2), using
- * the dst_pos of the latest ep_layout on this buffer.  smooth_scale is an fp32
- * [d] device vector or NULL; it must be NULL when cfg.smooth_rows == 0. */
+ * every routed pick into recv_x (plus recv_scale, token_scale in mode 2), to the
+ * receive rows of the latest ep_layout on this buffer.  smooth_scale is an fp32
+ * [d] device vector or NULL; it must be NULL when cfg.smooth_rows == 0.
+ * For T = B/P <= 256 the kernel derives those rows from the topk_idx passed to
+ * that ep_layout (which must still hold the same ids) instead of reading dst_pos,
+ * so it can run alongside the layout kernel; it finishes only after the layout
+ * kernel has.  Call it on the stream of that ep_layout, after it. */
 EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale,
                 ep_stream_t stream);
 
