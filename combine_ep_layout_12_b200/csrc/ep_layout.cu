@@ -131,15 +131,16 @@ __device__ __forceinline__ unsigned classify_ids(const int* ids, int k, int E, i
 }
 
 // Layout for small per-rank batches (T <= 256), with no dependency between CTAs.
-//  - CTA 0 (the count CTA) histograms every token's routed ids per (expert, rank)
-//    and the special ids, and writes recv_count, expert_count and expert_offset.
-//  - Every other CTA holds 8 warps; warp q handles the q-th 32-token chunk of a
-//    rank.  It counts, per expert, the rank's tokens before its chunk (read from
-//    L2; a token counts once per expert), sets one lane bit per routed id of its
-//    own tokens, and a token's slot is  before[g] + popc(mask[g] & lanemask_lt),
-//    i.e. its rank among the rank's tokens that routed to g, in token order.
-// Both halves only use order-independent shared-memory atomics, so the result is
-// deterministic.
+//  - CTA 0 (the count CTA) histograms every token's ids per expert id (routed and
+//    special) and writes expert_count and its exclusive prefix expert_offset.
+//  - Every other CTA holds whole ranks (8 / ceil(T/32) of them) with one warp per
+//    32-token chunk.  A warp sets, in shared memory, one lane bit per routed id of
+//    its tokens; after one barrier a token's slot is the popcount of the earlier
+//    chunks' masks of its rank plus popc(mask & lanemask_lt) of its own chunk,
+//    i.e. its rank among the rank's tokens that routed to g, in token order; the
+//    sum of its ranks' chunk popcounts per expert is recv_count.
+// Each warp reads only its own tokens' ids, and both halves use order-independent
+// shared-memory atomics, so the result is deterministic.
 template <int KM>
 __global__ void __launch_bounds__(256) layout_small_kernel(LayoutArgs a, int cpr) {
     extern __shared__ unsigned smem[];
@@ -151,12 +152,10 @@ __global__ void __launch_bounds__(256) layout_small_kernel(LayoutArgs a, int cpr
     pdl_launch_dependents();
 
     if (blockIdx.x == 0) {
-        int* cnt = reinterpret_cast<int*>(smem);     // [E][P]
-        int* spc = cnt + (size_t)E * P;               // [n_special]
-        int* ec = spc + a.n_special;                  // [E_tot]
-        int* wsum = ec + a.E_tot;                     // [32]
-        for (int i = threadIdx.x; i < E * P; i += blockDim.x) cnt[i] = 0;
-        for (int i = threadIdx.x; i < a.n_special; i += blockDim.x) spc[i] = 0;
+        // count CTA: picks per expert id over all tokens, then the exclusive prefix
+        int* ec = reinterpret_cast<int*>(smem);  // [E_tot]
+        int* wsum = ec + a.E_tot;                // [32]
+        for (int i = threadIdx.x; i < a.E_tot; i += blockDim.x) ec[i] = 0;
         __syncthreads();
         // four tokens per thread per pass, their id loads issued together
         const int stride = blockDim.x;
@@ -174,57 +173,33 @@ __global__ void __launch_bounds__(256) layout_small_kernel(LayoutArgs a, int cpr
             }
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-                const int t = t0 + b * stride;
-                if (t >= a.B) continue;
-                const int r = t / a.T;
+                if (t0 + b * stride >= a.B) continue;
                 const unsigned rb = classify_ids<KM>(ids[b], k, E, a.E_tot, err,
-                                                 [&](int sidx) { atomicAdd(&spc[sidx], 1); });
+                                                     [&](int sidx) { atomicAdd(&ec[E + sidx], 1); });
 #pragma unroll
                 for (int j = 0; j < KM; ++j)
-                    if (rb & (1u << j)) atomicAdd(&cnt[(size_t)ids[b][j] * P + r], 1);
+                    if (rb & (1u << j)) atomicAdd(&ec[ids[b][j]], 1);
             }
         }
         __syncthreads();
-        for (int i = threadIdx.x; i < E * P; i += blockDim.x) a.recv_count[i] = cnt[i];
-        for (int gg = threadIdx.x; gg < a.E_tot; gg += blockDim.x) {
-            int v = 0;
-            if (gg < E) {
-                for (int rr = 0; rr < P; ++rr) v += cnt[(size_t)gg * P + rr];
-            } else {
-                v = spc[gg - E];
-            }
-            ec[gg] = v;
-            a.expert_count[gg] = v;
-        }
+        for (int g = threadIdx.x; g < a.E_tot; g += blockDim.x) a.expert_count[g] = ec[g];
         report_err(&a.ws->err, err);
-        __syncthreads();
         block_exclusive_scan(ec, a.E_tot, a.expert_offset, wsum);
         return;
     }
 
-    // slot CTAs
+    // slot CTAs: whole ranks per CTA (8 / cpr of them), one warp per 32-token chunk
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = (blockIdx.x - 1) * (blockDim.x >> 5) + warp;  // chunk id
-    if (q >= P * cpr) return;  // no barrier below: whole warps leave together
-    const int r = q / cpr, c = q - r * cpr;
-    int* before = reinterpret_cast<int*>(smem) + (size_t)warp * E * 2;  // [E]
-    unsigned* mask = reinterpret_cast<unsigned*>(before + E);          // [E]
-    for (int g = lane; g < E; g += 32) {
-        before[g] = 0;
-        mask[g] = 0u;
-    }
-    __syncwarp();
-    unsigned ignore = 0;
-    for (int t = a.T * r + lane; t < a.T * r + c * 32; t += 32) {
-        int ids[KM];
-        load_token_ids<KM>(a.topk_idx, t, k, vec4, ids);
-        const unsigned rb = classify_ids<KM>(ids, k, E, a.E_tot, ignore, [](int) {});
-#pragma unroll
-        for (int j = 0; j < KM; ++j)
-            if (rb & (1u << j)) atomicAdd(&before[ids[j]], 1);
-    }
+    const int ranks_per_cta = 8 / cpr;
+    const int lr = warp / cpr, c = warp - lr * cpr;
+    const int r = (blockIdx.x - 1) * ranks_per_cta + lr;
+    const bool active = lr < ranks_per_cta && r < P;
+    unsigned* mask = reinterpret_cast<unsigned*>(smem);  // [8][E]
+    unsigned* my_mask = mask + (size_t)warp * E;
+    for (int g = lane; g < E; g += 32) my_mask[g] = 0u;
+    __syncthreads();
     const int t = a.T * r + c * 32 + lane;
-    const bool valid = c * 32 + lane < a.T;
+    const bool valid = active && c * 32 + lane < a.T;
     int ids[KM];
     unsigned rb = 0;
     if (valid) {
@@ -233,21 +208,33 @@ __global__ void __launch_bounds__(256) layout_small_kernel(LayoutArgs a, int cpr
     }
 #pragma unroll
     for (int j = 0; j < KM; ++j)
-        if (rb & (1u << j)) atomicOr(&mask[ids[j]], 1u << lane);
-    __syncwarp();
+        if (rb & (1u << j)) atomicOr(&my_mask[ids[j]], 1u << lane);
+    __syncthreads();
     if (valid) {
         const unsigned lt = lanemask_lt();
+        const unsigned* rank_masks = mask + (size_t)(lr * cpr) * E;
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
             if (j >= k) continue;
             int row = -1;
             if (rb & (1u << j)) {
                 const int g = ids[j];
-                row = g * P * a.M + r * a.M + before[g] + __popc(mask[g] & lt);
+                int before = 0;  // the rank's tokens in its earlier chunks that routed to g
+                for (int cc = 0; cc < c; ++cc) before += __popc(rank_masks[(size_t)cc * E + g]);
+                row = g * P * a.M + r * a.M + before + __popc(my_mask[g] & lt);
                 a.recv_src[row] = t;
             }
             a.dst_pos[(size_t)t * k + j] = row;
         }
+    }
+    // recv_count of this CTA's ranks: every chunk's popcount, per expert
+    for (int i = threadIdx.x; i < ranks_per_cta * E; i += blockDim.x) {
+        const int lrr = i / E, g = i - lrr * E;
+        const int rr = (blockIdx.x - 1) * ranks_per_cta + lrr;
+        if (rr >= P) continue;
+        int n = 0;
+        for (int cc = 0; cc < cpr; ++cc) n += __popc(mask[(size_t)(lrr * cpr + cc) * E + g]);
+        a.recv_count[(size_t)g * P + rr] = n;
     }
     // errors of the chunk's own tokens only (the count CTA reports the same bits)
     report_err(&a.ws->err, err);
@@ -410,8 +397,8 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     cudaGetDevice(&dev0);
     // small per-rank batches: count CTA + slot CTAs, no inter-CTA dependency
     const int cpr = (s.T + 31) / 32;
-    const size_t smem_count = sizeof(int) * ((size_t)s.E * s.P + s.n_special + s.E_tot + 32);
-    const size_t smem_slot = sizeof(int) * (size_t)8 * s.E * 2;
+    const size_t smem_count = sizeof(int) * ((size_t)s.E_tot + 32);
+    const size_t smem_slot = sizeof(int) * (size_t)8 * s.E;
     const size_t smem_small = smem_count > smem_slot ? smem_count : smem_slot;
     if (s.T <= 256 && smem_small <= budget) {
         if (dev0 < 16 && !attr_small[dev0]) {
@@ -434,8 +421,8 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         a1.B = s.B; a1.k = s.k; a1.P = s.P; a1.M = s.M; a1.E = s.E; a1.T = s.T;
         a1.n_special = s.n_special; a1.E_tot = s.E_tot;
         a1.warps = 8;
-        const int nchunks = s.P * cpr;
-        const int grid = 1 + (nchunks + 7) / 8;
+        const int ranks_per_cta = 8 / cpr;
+        const int grid = 1 + (s.P + ranks_per_cta - 1) / ranks_per_cta;
         cudaError_t e;
         if (s.k <= 2)
             e = launch_pdl(layout_small_kernel<2>, dim3(grid), dim3(256), smem_small, stream, a1, cpr);
