@@ -12,12 +12,12 @@ import torch
 
 from . import _binding as abi
 from ._binding import (EPError, ep_buffer_check, ep_buffer_create, ep_buffer_destroy,
-                       ep_buffer_size, ep_combine, ep_dispatch, ep_layout,
+                       ep_buffer_size, ep_combine, ep_dispatch, ep_layout, ep_layout_dispatch,
                        ep_layout_static_scratch, ep_status_str, make_config)
 
 __all__ = ["EPBuffer", "EPError", "abi", "ep_buffer_check", "ep_buffer_create",
            "ep_buffer_destroy", "ep_buffer_size", "ep_combine", "ep_dispatch", "ep_layout",
-           "ep_layout_static_scratch", "ep_status_str", "make_config"]
+           "ep_layout_dispatch", "ep_layout_static_scratch", "ep_status_str", "make_config"]
 
 
 def _ptr(t):
@@ -107,6 +107,15 @@ class EPBuffer:
         if smooth_scale is not None:
             _need(smooth_scale, "smooth_scale", torch.float32, (c.d,), self.device)
         ep_dispatch(self.handle, _ptr(x), _ptr(smooth_scale), _stream(stream))
+
+    def layout_dispatch(self, topk_idx, x, smooth_scale=None, stream=None):
+        """layout(topk_idx) then dispatch(x), as one call (one grid when T <= 128)."""
+        c = self.cfg
+        _need(topk_idx, "topk_idx", torch.int32, (c.B, c.k), self.device)
+        _need(x, "x", torch.bfloat16, (c.B, c.d), self.device)
+        if smooth_scale is not None:
+            _need(smooth_scale, "smooth_scale", torch.float32, (c.d,), self.device)
+        ep_layout_dispatch(self.handle, _ptr(topk_idx), _ptr(x), _ptr(smooth_scale), _stream(stream))
 
     def combine(self, expert_out, topk_idx, topk_weights, ori_x=None, a1=None, a2=None, v=None,
                 y=None, stream=None):

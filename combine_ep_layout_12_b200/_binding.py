@@ -63,11 +63,13 @@ def lib():
     L.ep_buffer_destroy.argtypes = [vp]
     L.ep_layout.argtypes = [vp, vp, vp]
     L.ep_dispatch.argtypes = [vp, vp, vp, vp]
+    L.ep_layout_dispatch.argtypes = [vp, vp, vp, vp, vp]
     L.ep_combine.argtypes = [vp] * 10
     L.ep_buffer_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.ep_layout_static_scratch.argtypes = [ctypes.POINTER(ep_config)] + [vp] * 8
     for f in (L.ep_buffer_size, L.ep_buffer_create, L.ep_buffer_destroy, L.ep_layout,
-              L.ep_dispatch, L.ep_combine, L.ep_buffer_check, L.ep_layout_static_scratch):
+              L.ep_dispatch, L.ep_layout_dispatch, L.ep_combine, L.ep_buffer_check,
+              L.ep_layout_static_scratch):
         f.restype = i
     L.ep_status_str.argtypes = [i]
     L.ep_status_str.restype = ctypes.c_char_p
@@ -112,6 +114,11 @@ def ep_layout(handle, topk_idx, stream=0):
 
 def ep_dispatch(handle, x, smooth_scale=None, stream=0):
     _check(lib().ep_dispatch(handle, x, smooth_scale, stream), "ep_dispatch")
+
+
+def ep_layout_dispatch(handle, topk_idx, x, smooth_scale=None, stream=0):
+    _check(lib().ep_layout_dispatch(handle, topk_idx, x, smooth_scale, stream),
+           "ep_layout_dispatch")
 
 
 def ep_combine(handle, expert_out, topk_idx, topk_weights, ori_x, a1, a2, v, y, stream=0):

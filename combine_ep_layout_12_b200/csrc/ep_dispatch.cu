@@ -16,245 +16,28 @@
 // to each of the token's k receive rows with 16-byte stores.  The read happens
 // once per token; the k writes are the bulk of the traffic.
 #include "ep_internal.cuh"
+#include "ep_dispatch_dev.cuh"
 
 namespace ep {
 namespace {
 
-constexpr int kSelfRowsMaxT = 256;
-
-struct DispatchArgs {
-    const uint16_t* x;       // [B][d] bf16
-    const float* smooth;     // [d] or null
-    const int32_t* dst_pos;  // [B][k]
-    const int32_t* topk_idx; // [B][k]; read instead of dst_pos when self_rows
-    int self_rows;           // compute the receive rows here (small T) instead of reading dst_pos
-    int T, P, M, E;
-    void* recv_x;            // [rows][d] int8 or bf16
-    float* recv_scale;       // [rows]
-    float* token_scale;      // [B]
-    unsigned* err;
-    long long rows;
-    int d, k;
-};
-
-// Receive rows of token t computed from the routing alone (used when T is small):
-// the slot of a routed id g is the number of earlier tokens of the same rank that
-// routed to g (a token counts once), which is exactly the slot the layout kernel
-// assigns.  The earlier tokens' ids come from L2 while the x row load is in
-// flight.  s_g, s_cnt: k-entry shared arrays.  Ends with s_rows published.
-__device__ void compute_rows(const DispatchArgs& a, int t, int* s_rows, int* s_g, int* s_cnt) {
-    const int k = a.k;
-    if (threadIdx.x < k) {
-        const int j = threadIdx.x;
-        const int g = a.topk_idx[(size_t)t * k + j];
-        bool routed = g >= 0 && g < a.E;
-        for (int jj = 0; jj < j; ++jj)
-            if (a.topk_idx[(size_t)t * k + jj] == g) routed = false;  // repeated id: dropped
-        s_g[j] = routed ? g : -1;
-        s_cnt[j] = 0;
-    }
-    __syncthreads();
-    const int r = t / a.T;
-    for (int tt = r * a.T + (int)threadIdx.x; tt < t; tt += blockDim.x) {
-        const int32_t* ids = a.topk_idx + (size_t)tt * k;
-        unsigned hit = 0;
-        for (int jj = 0; jj < k; ++jj) {
-            const int v = __ldg(ids + jj);
-            for (int j = 0; j < k; ++j) {
-                const int g = s_g[j];
-                if (g >= 0 && v == g) hit |= 1u << j;
-            }
-        }
-        while (hit) {
-            const int j = __ffs(hit) - 1;
-            hit &= hit - 1;
-            atomicAdd(&s_cnt[j], 1);
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < k) {
-        const int g = s_g[threadIdx.x];
-        s_rows[threadIdx.x] = g >= 0 ? g * a.P * a.M + r * a.M + s_cnt[threadIdx.x] : -1;
-    }
-}
-
-// Receive rows of token t into shared memory; out-of-range rows are skipped and flagged.
-__device__ __forceinline__ void load_rows(const DispatchArgs& a, int t, int* s_rows) {
-    unsigned bad = 0;
-    if (threadIdx.x < a.k) {
-        int row = a.dst_pos[(size_t)t * a.k + threadIdx.x];
-        if (row < -1 || (long long)row >= a.rows) {
-            bad = EP_ERRBIT_ROW_RANGE;
-            row = -1;
-        }
-        s_rows[threadIdx.x] = row;
-    }
-    if (threadIdx.x < 32) report_err(a.err, bad);
-}
-
-// x_fp32 of the two bf16 halves of one 32-bit word, times the smooth scale when given.
-__device__ __forceinline__ void xf_pair(uint32_t w, const float* ss, int i, float& lo, float& hi) {
-    lo = bf16lo(w);
-    hi = bf16hi(w);
-    if (ss) {
-        lo = __fmul_rn(lo, ss[i]);
-        hi = __fmul_rn(hi, ss[i + 1]);
-    }
-}
-
-// CastToInt8 of x_fp32 * s: round half to even, saturate.
-__device__ __forceinline__ uint32_t q8(float xf, float s) {
-    const int q = min(127, max(-128, __float2int_rn(__fmul_rn(xf, s))));
-    return (uint32_t)(q & 0xff);
-}
-
-// quant_mode 2: a unit is 16 elements (two 16-byte bf16 loads -> one 16-byte int8 store).
+// Dispatch kernels.  With self_rows the kernel needs nothing the layout kernel
+// writes, so it runs alongside it and waits for it only before exiting (so that
+// whatever follows on the stream sees a finished layout); otherwise it waits first.
 template <int U>
 __global__ void __launch_bounds__(256) dispatch_int8_kernel(DispatchArgs a) {
-    __shared__ int s_rows[kMaxK];
-    __shared__ float s_red[32];
-    const int t = blockIdx.x;
-    const int nunits = a.d >> 4;
-    const int NT = blockDim.x;
-
-    __shared__ int s_g[kMaxK], s_cnt[kMaxK];
-    // With self_rows the kernel needs nothing the layout kernel writes, so it
-    // runs alongside it and waits for it only before exiting (so that whatever
-    // follows on the stream sees a finished layout); otherwise it waits first.
     if (!a.self_rows) pdl_wait();
     pdl_launch_dependents();
-
-    const uint4* xrow = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d);
-    uint4 raw[U][2];
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-        const int u = threadIdx.x + i * NT;
-        if (u < nunits) {
-            raw[i][0] = ld_stream_v4(xrow + 2 * u);
-            raw[i][1] = ld_stream_v4(xrow + 2 * u + 1);
-        } else {
-            raw[i][0] = make_uint4(0, 0, 0, 0);
-            raw[i][1] = make_uint4(0, 0, 0, 0);
-        }
-    }
-    if (a.self_rows)
-        compute_rows(a, t, s_rows, s_g, s_cnt);
-    else
-        load_rows(a, t, s_rows);
-
-    // x_fp32 = fp32(x) * smooth; absmax over the row
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-        const int u = threadIdx.x + i * NT;
-        if (u >= nunits) continue;
-        const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
-                               raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
-        const float* ss = a.smooth ? a.smooth + 16 * u : nullptr;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float lo, hi;
-            xf_pair(w[e], ss, 2 * e, lo, hi);
-            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
-    __syncthreads();  // also publishes s_rows
-    if (threadIdx.x < 32) {
-        float m = threadIdx.x < (NT >> 5) ? s_red[threadIdx.x] : 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (threadIdx.x == 0) s_red[0] = m;
-    }
-    __syncthreads();
-    amax = s_red[0];
-
-    const float s = __fdiv_rn(127.0f, amax);
-    const bool degenerate = (amax == 0.0f) || isinf(s);
-    const float inv = degenerate ? 0.0f : __fdiv_rn(1.0f, s);
-    int8_t* out = reinterpret_cast<int8_t*>(a.recv_x);
-
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-        const int u = threadIdx.x + i * NT;
-        if (u >= nunits) continue;
-        const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
-                               raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
-        const float* ss = a.smooth ? a.smooth + 16 * u : nullptr;
-        uint32_t word[4];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            float x0, x1, x2, x3;
-            xf_pair(w[2 * h], ss, 4 * h, x0, x1);
-            xf_pair(w[2 * h + 1], ss, 4 * h + 2, x2, x3);
-            word[h] = degenerate ? 0u
-                                 : (q8(x0, s) | (q8(x1, s) << 8) | (q8(x2, s) << 16) | (q8(x3, s) << 24));
-        }
-        const uint4 v = make_uint4(word[0], word[1], word[2], word[3]);
-        for (int j = 0; j < a.k; ++j) {
-            const int row = s_rows[j];
-            if (row >= 0) st_v4(out + (size_t)row * a.d + 16 * u, v);
-        }
-    }
-    if (threadIdx.x < a.k) {
-        const int row = s_rows[threadIdx.x];
-        if (row >= 0) a.recv_scale[row] = inv;
-    }
-    if (threadIdx.x == 0) a.token_scale[t] = inv;
+    dispatch_int8_body<U>(a, blockIdx.x);
     if (a.self_rows) pdl_wait();
 }
 
-// quant_mode 0: bf16 rows copied as they are; a unit is one 16-byte vector.
 template <int U>
 __global__ void __launch_bounds__(256) dispatch_bf16_kernel(DispatchArgs a) {
-    __shared__ int s_rows[kMaxK];
-    const int t = blockIdx.x;
-    const int nvec = a.d >> 3;
-    const int NT = blockDim.x;
-
-    __shared__ int s_g[kMaxK], s_cnt[kMaxK];
     if (!a.self_rows) pdl_wait();
     pdl_launch_dependents();
-
-    const uint4* xrow = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.d);
-    uint4 raw[U];
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-        const int u = threadIdx.x + i * NT;
-        raw[i] = (u < nvec) ? ld_stream_v4(xrow + u) : make_uint4(0, 0, 0, 0);
-    }
-    if (a.self_rows)
-        compute_rows(a, t, s_rows, s_g, s_cnt);
-    else
-        load_rows(a, t, s_rows);
-    __syncthreads();
-    uint4* out = reinterpret_cast<uint4*>(a.recv_x);
-#pragma unroll
-    for (int i = 0; i < U; ++i) {
-        const int u = threadIdx.x + i * NT;
-        if (u >= nvec) continue;
-        for (int j = 0; j < a.k; ++j) {
-            const int row = s_rows[j];
-            if (row >= 0) st_v4(out + (size_t)row * nvec + u, raw[i]);
-        }
-    }
+    dispatch_bf16_body<U>(a, blockIdx.x);
     if (a.self_rows) pdl_wait();
-}
-
-int pick_units(int n, int max_u, int* U, int* NT) {
-    // Smallest power-of-two U <= max_u with ceil(n / U) <= 128 threads: small CTAs
-    // (and few registers) so that a decode batch of ~1000 tokens is resident in one
-    // wave.  Wider rows fall back to up to 256 threads.
-    int u = 1;
-    while (u < max_u && (n + u - 1) / u > 128) u *= 2;
-    int nt = (n + u - 1) / u;
-    nt = ((nt + 31) / 32) * 32;
-    if (nt > 256) return EP_ERR_UNSUPPORTED;
-    *U = u;
-    *NT = nt;
-    return EP_OK;
 }
 
 }  // namespace
@@ -262,22 +45,7 @@ int pick_units(int n, int max_u, int* U, int* NT) {
 int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
                     const float* smooth, const int32_t* topk_idx, cudaStream_t stream) {
     if (s.B == 0) return EP_OK;
-    DispatchArgs a;
-    a.x = x;
-    a.smooth = smooth;
-    a.dst_pos = p.dst_pos;
-    a.recv_x = p.recv_x;
-    a.recv_scale = p.recv_scale;
-    a.token_scale = p.token_scale;
-    a.err = &reinterpret_cast<WsHeader*>(p.workspace)->err;
-    a.rows = s.rows;
-    a.d = s.d;
-    a.k = s.k;
-    a.topk_idx = topk_idx;
-    a.T = s.T;
-    a.P = s.P;
-    a.M = s.M;
-    a.E = s.E;
+    DispatchArgs a = make_dispatch_args(s, p, x, smooth, topk_idx);
     // Small batches per rank: each CTA derives its rows from the routing itself
     // (at most kSelfRowsMaxT earlier tokens to scan), so dispatch overlaps layout.
     a.self_rows = (topk_idx != nullptr && s.T <= kSelfRowsMaxT) ? 1 : 0;

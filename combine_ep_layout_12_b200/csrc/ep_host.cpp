@@ -57,8 +57,8 @@ void fill_sizes(const ep_config* c, ep_buffer_sizes* s) {
     s->recv_x = rows * (size_t)c->d * esz;
     s->recv_scale = c->quant_mode == 2 ? 4 * rows : 0;
     s->token_scale = c->quant_mode == 2 ? 4 * (size_t)c->B : 0;
-    const size_t ws = sizeof(ep::WsHeader) + 4 * (size_t)c->P * n_special;
-    s->workspace = (ws + 255) & ~(size_t)255;
+    (void)n_special;
+    s->workspace = ep::workspace_bytes(ep::make_shape(*c));
 }
 
 bool ptr_ok(const void* p, size_t size) { return size == 0 || (p != nullptr && aligned16(p)); }
@@ -122,6 +122,20 @@ int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale, ep
     if (smooth_scale && c.quant_mode != 2) return EP_ERR_INVALID_ARG;
     return ep::launch_dispatch(ep::make_shape(c), buf->ptrs, x, smooth_scale, buf->last_topk_idx,
                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx, const uint16_t* x,
+                       const float* smooth_scale, ep_stream_t stream) {
+    if (!buf) return EP_ERR_INVALID_ARG;
+    const ep_config& c = buf->cfg;
+    if (c.B > 0 && (!topk_idx || !aligned4(topk_idx))) return EP_ERR_INVALID_ARG;
+    if (c.B > 0 && (!x || !aligned16(x))) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && (c.smooth_rows == 0 || !aligned16(smooth_scale))) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && c.quant_mode != 2) return EP_ERR_INVALID_ARG;
+    const int st = ep::launch_layout_dispatch(ep::make_shape(c), buf->ptrs, topk_idx, x, smooth_scale,
+                                              reinterpret_cast<cudaStream_t>(stream));
+    buf->last_topk_idx = st == EP_OK ? topk_idx : nullptr;
+    return st;
 }
 
 int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,

@@ -42,6 +42,15 @@ inline Shape make_shape(const ep_config& c) {
     return s;
 }
 
+// Workspace layout: WsHeader, then the multi-CTA layout's per-rank special
+// counts [P][n_special].
+inline size_t workspace_layout_bytes(const Shape& s) {
+    return sizeof(WsHeader) + 4 * (size_t)s.P * s.n_special;
+}
+inline size_t workspace_bytes(const Shape& s) {
+    return (workspace_layout_bytes(s) + 255) & ~(size_t)255;
+}
+
 // Host launchers (one per kernel family); each returns an EP_* status.
 int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
                   cudaStream_t stream);
@@ -49,6 +58,10 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
 // its receive rows itself for small per-rank batches); may be null.
 int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
                     const float* smooth, const int32_t* topk_idx, cudaStream_t stream);
+// Layout and dispatch of the same routing in one grid when the batch per rank is
+// small (T <= 128, k <= 8); otherwise the two launches above, in order.
+int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
+                           const uint16_t* x, const float* smooth, cudaStream_t stream);
 int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
                    const int32_t* topk_idx, const float* topk_weights, const uint16_t* ori_x,
                    const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,

@@ -73,7 +73,15 @@ class Pipeline:
                                 ori_x=dev_inp["x"], a1=dev_inp.get("a1"), a2=dev_inp.get("a2"),
                                 v=dev_inp.get("v"), y=self.y, stream=stream)
 
-    def step(self, dev_inp, stream=None):
-        self.layout(dev_inp, stream)
-        self.dispatch(dev_inp, stream)
+    def layout_dispatch(self, dev_inp, stream=None):
+        self.buf.layout_dispatch(dev_inp["topk_idx"], dev_inp["x"], dev_inp.get("smooth"),
+                                 stream=stream)
+
+    def step(self, dev_inp, stream=None, fused=True):
+        """layout -> dispatch -> combine; fused=True issues the first two as one call."""
+        if fused:
+            self.layout_dispatch(dev_inp, stream)
+        else:
+            self.layout(dev_inp, stream)
+            self.dispatch(dev_inp, stream)
         return self.combine(dev_inp, stream)

@@ -167,6 +167,15 @@ EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, ep_stream_t stream
 EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale,
                 ep_stream_t stream);
 
+/* ep_layout followed by ep_dispatch on the same stream, as one call: same
+ * outputs, bit for bit.  When T = B/P <= 128 and k <= 8 both run in a single
+ * grid (the layout in its first CTAs, one token's dispatch in each of the
+ * others, which derives its receive rows from the routing itself), saving one
+ * kernel launch on the critical path; otherwise the two kernels are launched in
+ * order.  Arguments as for ep_layout and ep_dispatch. */
+EP_API int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx, const uint16_t* x,
+                              const float* smooth_scale, ep_stream_t stream);
+
 /* Weighted combine into y (bf16 [B][d], device).  expert_out: bf16 [E*P*M][d]
  * receive-layout expert outputs (may alias recv_x when quant_mode is 0);
  * topk_idx int32 [B][k] and topk_weights fp32 [B][k] as given to ep_layout;

@@ -47,16 +47,20 @@ def need_bytes(w, separate_expert_out):
     return total
 
 
-def full_check(w, dev, inp=None, tokens=None, sample_picks=None, separate=True):
-    """Layout + dispatch + combine of one workload against the oracle."""
+def full_check(w, dev, inp=None, tokens=None, sample_picks=None, separate=True, fused=False):
+    """Layout + dispatch + combine of one workload against the oracle.  fused: issue
+    layout and dispatch as the single ep_layout_dispatch call."""
     inp = inp if inp is not None else wl.generate(w)
     if need_bytes(w, separate) > free_bytes() - (4 << 30):
         pytest.skip("%s needs %.1f GB of device memory" % (w.name, need_bytes(w, separate) / 1e9))
     dev_inp = runner.to_device(inp, dev)
     pipe = runner.Pipeline(w, dev, alias_expert_out=not separate)
     rep = gp.Report()
-    pipe.layout(dev_inp)
-    pipe.dispatch(dev_inp)
+    if fused:
+        pipe.layout_dispatch(dev_inp)
+    else:
+        pipe.layout(dev_inp)
+        pipe.dispatch(dev_inp)
     err = pipe.buf.check()
     ref = oracle.layout(gp.ocfg(w), inp["topk_idx"])
     rep.check(err == ref["err"], "%s: device error bits %#x, oracle %#x" % (w.name, err, ref["err"]))
@@ -157,6 +161,40 @@ def test_prefill(dev):
     # sampled tokens against the oracle with softmax weights
     tokens = np.sort(rng.choice(w.B, 512, replace=False))
     gp.check_combine(rep, w, pipe, inp, dev_inp, ref, tokens=tokens)
+    rep.assert_ok()
+
+
+# ----------------------------------------------------------------------------- fused call
+
+
+@pytest.mark.parametrize("name", ["tiny_q0", "tiny_q2", "decode", "sweep_T1_q2", "sweep_T16_q0",
+                                  "sweep_T64_q2", "sweep_T256_q0", "skewed"])
+def test_layout_dispatch_one_call(dev, name):
+    """ep_layout_dispatch (one grid when T <= 128 and k <= 8, else two launches)
+    against the oracle: identical to ep_layout followed by ep_dispatch."""
+    full_check(wl.get(name), dev, fused=True)
+
+
+def test_layout_dispatch_one_call_dirty(dev):
+    w = wl.Workload("ragged_fused", B=111, d=272, k=3, P=3, M=40, E=9, n_zero=1, n_copy=1,
+                    n_const=1, quant_mode=2, smooth="rand", seed=5)
+    inp = wl.generate(w)
+    rng = np.random.default_rng(6)
+    idx = np.stack([rng.permutation(w.E_tot)[:w.k] for _ in range(w.B)]).astype(np.int32)
+    idx[2, 0] = -1
+    idx[5, 1] = w.E_tot
+    idx[11] = [3, 7, 3]
+    inp["topk_idx"] = idx
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev, alias_expert_out=False)
+    pipe.layout_dispatch(dev_inp)
+    err = pipe.buf.check()
+    ref = oracle.layout(gp.ocfg(w), idx)
+    assert err == ref["err"] == (oracle.ERR_BAD_ID | oracle.ERR_DUP_ID)
+    rep = gp.Report()
+    gp.check_layout(rep, w, pipe, ref)
+    gp.check_dispatch(rep, w, pipe, inp, ref)
+    gp.check_combine(rep, w, pipe, inp, dev_inp, ref)
     rep.assert_ok()
 
 
