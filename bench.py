@@ -61,6 +61,9 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle baseline")
+    p.add_argument("--sweep", default=None,
+                   help="comma-separated workloads or 'all': per-workload table instead of the JSON line")
+    p.add_argument("--sweep-out", default=None, help="where --sweep writes its JSON document")
     return p.parse_args(argv)
 
 
@@ -319,10 +322,119 @@ def config_dict(w, args):
 # ----------------------------------------------------------------------------- our arm
 
 
+class Workbench:
+    """Device buffers of one workload, rotated over `R` sets, plus the CUDA graphs
+    that time it: steps (ep_layout_dispatch -> ep_combine) and per-kernel loops."""
+
+    def __init__(self, w, inp, device, stream, max_sets, flush_mb):
+        import torch
+        from combine_ep_layout_12_b200 import metrics, runner
+        self.w, self.device, self.stream = w, device, stream
+        set_bytes = w.rows * w.d * (1 if w.quant_mode == 2 else 2) + w.rows * 12 + 4 * w.B * w.d
+        if w.quant_mode == 2:
+            set_bytes += w.rows * w.d * 2
+        free = torch.cuda.mem_get_info(device)[0]
+        if set_bytes > 0.9 * free:
+            raise MemoryError("%s needs %.1f GB of device memory, %.1f GB free"
+                              % (w.name, set_bytes / 1e9, free / 1e9))
+        # consecutive steps touch disjoint memory when two or more sets fit; with
+        # one set, L2 is flushed between steps instead
+        self.R = int(max(1, min(max_sets, (0.8 * free) // max(set_bytes, 1))))
+        self.sets = []
+        for _ in range(self.R):
+            dev_inp = runner.to_device(inp, device)
+            pipe = runner.Pipeline(w, device)
+            with torch.cuda.stream(stream):
+                pipe.layout(dev_inp, stream)
+                pipe.dispatch(dev_inp, stream)
+            stream.synchronize()
+            assert pipe.buf.check(stream) == 0, "device error bits set"
+            dp = pipe.buf.dst_pos
+            rows = dp[dp >= 0].long()
+            if w.quant_mode == 2:  # identity expert: expert_out rows = dequantized receive rows
+                deq = pipe.buf.recv_x[rows].float() * pipe.buf.recv_scale[rows].unsqueeze(1)
+                pipe.expert_out[rows] = deq.to(torch.bfloat16)
+            self.sets.append((pipe, dev_inp))
+        torch.cuda.synchronize(device)
+        self.n_routed = int((self.sets[0][0].buf.dst_pos >= 0).sum().item())
+        _, b_sp = metrics.routing_counts(w, inp["topk_idx"], self.n_routed)
+        self.kbytes = metrics.kernel_bytes(w, self.n_routed, b_sp, smooth=inp["smooth"] is not None)
+        self.step_bytes = sum(self.kbytes.values())
+        self.flush = None
+        if self.R == 1 and flush_mb:
+            self.flush = torch.empty(flush_mb << 20, dtype=torch.uint8, device=device)
+        self.S = 2 * self.R if self.R > 1 else 1
+        units = w.d // 16 if w.quant_mode == 2 else w.d // 8
+        # ep_layout_dispatch runs as one grid when T <= 128, k <= 8 and a row fits 128 threads
+        self.one_grid = w.B > 0 and w.T <= 128 and w.k <= 8 and units <= 1024
+        self.launches_per_step = 2 if self.one_grid else 3
+
+    def capture(self, fn):
+        import torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream):
+            fn()
+        return g
+
+    def steps_graph(self, n):
+        def body():
+            for i in range(n):
+                if self.flush is not None:
+                    self.flush.zero_()
+                p, d = self.sets[i % self.R]
+                p.step(d, self.stream)
+        return self.capture(body)
+
+    def kernel_graph(self, names):
+        def body():
+            for i in range(self.S):
+                p, d = self.sets[i % self.R]
+                for name in names:
+                    if self.flush is not None:
+                        self.flush.zero_()
+                    getattr(p, name)(d, self.stream)
+        return self.capture(body)
+
+    def replay(self, g, n):
+        """Replays g n times between two CUDA events; returns milliseconds."""
+        import torch
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            a.record(self.stream)
+            for _ in range(n):
+                g.replay()
+            b.record(self.stream)
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    def kernel_times(self, launches):
+        """Per-launch milliseconds of each kernel and of the one-call layout+dispatch,
+        from graphs of S back-to-back launches replayed about `launches / S` times.
+        With one buffer set each launch is preceded by an L2 flush inside the graph;
+        that memset is timed too and subtracted."""
+        graphs = {"layout": ["layout"], "dispatch": ["dispatch"], "combine": ["combine"],
+                  "layout+dispatch": ["layout", "dispatch"], "layout_dispatch": ["layout_dispatch"]}
+        n_rep = max(1, launches // self.S)
+        out = {}
+        for key, names in graphs.items():
+            g = self.kernel_graph(names)
+            self.replay(g, 1)
+            out[key] = self.replay(g, n_rep) / (n_rep * self.S)
+        if self.flush is not None:
+            def fbody():
+                for _ in range(self.S):
+                    self.flush.zero_()
+            g = self.capture(fbody)
+            self.replay(g, 1)
+            f = self.replay(g, n_rep) / (n_rep * self.S)
+            out = {k: v - f * (2 if k == "layout+dispatch" else 1) for k, v in out.items()}
+        return out, n_rep
+
+
 def run_ours(args):
     import torch
     from combine_ep_layout_12_b200 import build as ep_build
-    from combine_ep_layout_12_b200 import metrics, runner
+    from combine_ep_layout_12_b200 import runner
     from combine_ep_layout_12_b200 import workloads as wl
 
     world, rank, local = dist_env()
@@ -332,103 +444,30 @@ def run_ours(args):
     device = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
     ep_build.build()
+    if args.sweep:
+        return run_sweep(args, device)
 
     w = wl.get(args.workload)
     inp = wl.generate(w)
     stream = torch.cuda.Stream(device)
-
-    # Buffer sets used in rotation, so that consecutive steps touch disjoint memory
-    # and the second use of a set finds nothing of it left in L2; when memory does
-    # not allow two sets, one set with an L2 flush between steps.
-    set_bytes = w.rows * w.d * (1 if w.quant_mode == 2 else 2) + w.rows * 12 + 4 * w.B * w.d
-    if w.quant_mode == 2:
-        set_bytes += w.rows * w.d * 2
-    free = torch.cuda.mem_get_info(device)[0]
-    R = int(max(1, min(args.sets, (0.8 * free) // max(set_bytes, 1))))
-    sets = []
-    for _ in range(R):
-        dev_inp = runner.to_device(inp, device)
-        pipe = runner.Pipeline(w, device)
-        with torch.cuda.stream(stream):
-            pipe.layout(dev_inp, stream)
-            pipe.dispatch(dev_inp, stream)
-        stream.synchronize()
-        assert pipe.buf.check(stream) == 0, "device error bits set"
-        dp = pipe.buf.dst_pos
-        rows = dp[dp >= 0].long()
-        if w.quant_mode == 2:  # identity expert: expert_out rows = dequantized receive rows
-            deq = pipe.buf.recv_x[rows].float() * pipe.buf.recv_scale[rows].unsqueeze(1)
-            pipe.expert_out[rows] = deq.to(torch.bfloat16)
-        sets.append((pipe, dev_inp))
-    torch.cuda.synchronize(device)
-    n_routed = int((sets[0][0].buf.dst_pos >= 0).sum().item())
-    _, b_sp = metrics.routing_counts(w, inp["topk_idx"], n_routed)
-    kbytes = metrics.kernel_bytes(w, n_routed, b_sp, smooth=inp["smooth"] is not None)
-    step_bytes = sum(kbytes.values())
-    flush = None
-    if R == 1 and args.flush_mb:
-        flush = torch.empty(args.flush_mb << 20, dtype=torch.uint8, device=device)
-
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            fn()
-        return g
-
-    # one graph per set holding one step (layout -> dispatch -> combine, with
-    # programmatic-launch edges between the kernels): the per-step latency loop
-    step_graphs = [capture(lambda p=p, d=d: p.step(d, stream)) for p, d in sets]
-    # graphs of S consecutive steps over the sets: the timed throughput loop
-    S = 2 * R if R > 1 else 1
+    wb = Workbench(w, inp, device, stream, args.sets, args.flush_mb)
+    R, S, sets = wb.R, wb.S, wb.sets
     K = args.steps
 
-    def steps_body(n):
-        def body():
-            for i in range(n):
-                if flush is not None:
-                    flush.zero_()
-                p, d = sets[i % R]
-                p.step(d, stream)
-        return body
-    multi_graph = capture(steps_body(S))
-    rem_graph = capture(steps_body(K % S)) if K % S else None
-    # one graph per kernel holding S back-to-back launches of it over the sets
-    kern_graphs = {}
-    for name in ("layout", "dispatch", "combine"):
-        def body(name=name):
-            for i in range(S):
-                p, d = sets[i % R]
-                getattr(p, name)(d, stream)
-        kern_graphs[name] = capture(body)
+    # one graph per set holding one step: warm-up and the per-step latency loop;
+    # graphs of S consecutive steps over the sets: the timed throughput loop
+    step_graphs = [wb.capture(lambda p=p, d=d: p.step(d, stream)) for p, d in sets]
+    multi_graph = wb.steps_graph(S)
+    rem_graph = wb.steps_graph(K % S) if K % S else None
 
-    def pair_body():
-        for i in range(S):
-            p, d = sets[i % R]
-            p.layout(d, stream)
-            p.dispatch(d, stream)
-    kern_graphs["layout+dispatch"] = capture(pair_body)
-
-    def fused_body():
-        for i in range(S):
-            p, d = sets[i % R]
-            p.layout_dispatch(d, stream)
-    kern_graphs["layout_dispatch"] = capture(fused_body)
-
-    def replay(g):
-        if flush is not None:
-            flush.zero_()
-        g.replay()
-
-    # warm-up: W steps (single-step graphs), then one replay of every other graph
-    # so that each is uploaded before it is timed
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            replay(step_graphs[i % R])
+            if wb.flush is not None:
+                wb.flush.zero_()
+            step_graphs[i % R].replay()
         multi_graph.replay()
         if rem_graph is not None:
             rem_graph.replay()
-        for g in kern_graphs.values():
-            replay(g)
     stream.synchronize()
 
     clocks = ClockSampler(device.index if device.index is not None else 0)
@@ -448,35 +487,27 @@ def run_ours(args):
             rem_graph.replay()
         t1_ev.record(stream)
     torch.cuda.synchronize(device)
-    t_wall1 = time.perf_counter()
     barrier(dist, device)
     local_s = t0_ev.elapsed_time(t1_ev) / 1e3
+    if wb.flush is not None:  # the flush memsets are inside the step graphs: take them out
+        fg = wb.capture(lambda: [wb.flush.zero_() for _ in range(S)])
+        wb.replay(fg, 1)
+        local_s -= wb.replay(fg, max(1, K // S)) / 1e3 * (K / (max(1, K // S) * S))
 
     # per-step latency: single-step graph replays, CUDA events around each
     n_lat = min(K, 500)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_lat)]
     with torch.cuda.stream(stream):
         for i in range(n_lat):
-            if flush is not None:
-                flush.zero_()
+            if wb.flush is not None:
+                wb.flush.zero_()
             ev[2 * i].record(stream)
             step_graphs[i % R].replay()
             ev[2 * i + 1].record(stream)
     torch.cuda.synchronize(device)
     step_ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n_lat)]
 
-    # per-kernel durations: S launches per graph replay, back to back
-    n_rep = max(1, K // S)
-    kern_ms = {}
-    with torch.cuda.stream(stream):
-        for name, g in kern_graphs.items():
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(n_rep):
-                replay(g)
-            b.record(stream)
-            b.synchronize()
-            kern_ms[name] = a.elapsed_time(b) / (n_rep * S)
+    kern_ms, n_rep = wb.kernel_times(K)
     t_wall2 = time.perf_counter()
     clocks.mark(t_wall0, t_wall2)
     time.sleep(0.03)
@@ -484,7 +515,7 @@ def run_ours(args):
     for p, _ in sets:
         assert p.buf.check(stream) == 0, "device error bits set during the timed steps"
 
-    job_s, job_bytes = aggregate(dist, local_s, float(step_bytes * K), device)
+    job_s, job_bytes = aggregate(dist, local_s, float(wb.step_bytes * K), device)
     _, job_tokens = aggregate(dist, local_s, float(w.B * K), device)
     value = job_bytes / job_s / 1e9
 
@@ -493,8 +524,8 @@ def run_ours(args):
     tot = sum(kern_ms[n] for n in ("layout", "dispatch", "combine"))
     for name in ("layout", "dispatch", "combine"):
         ms = kern_ms[name]
-        ach = kbytes[name] / (ms * 1e-3) / 1e9
-        kernels[name] = {"us": 1e3 * ms, "bytes": kbytes[name], "achieved_gbs": ach,
+        ach = wb.kbytes[name] / (ms * 1e-3) / 1e9
+        kernels[name] = {"us": 1e3 * ms, "bytes": wb.kbytes[name], "achieved_gbs": ach,
                          "frac_of_measured": ach / peak, "frac_of_8tbs": ach / SPEC_HBM_GBS,
                          "share": ms / tot}
     dom = max(("dispatch", "combine", "layout"), key=lambda n: kernels[n]["share"])
@@ -504,7 +535,7 @@ def run_ours(args):
                 "peak_source": ("%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peak_kind)
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "frac_of_8tbs_spec": kernels[dom]["achieved_gbs"] / SPEC_HBM_GBS,
-                "algorithmic_bytes": kbytes[dom],
+                "algorithmic_bytes": wb.kbytes[dom],
                 "duration": "CUDA events around graphs of %d back-to-back launches, %d replays" % (S, n_rep)}
 
     # end to end through the public API with host buffers (eager calls, no graph)
@@ -523,8 +554,8 @@ def run_ours(args):
         with torch.cuda.stream(stream):
             for i in range(Ke):
                 p, d = sets[i % R]
-                if flush is not None:
-                    flush.zero_()
+                if wb.flush is not None:
+                    wb.flush.zero_()
                 e0[i].record(stream)
                 for n in names:
                     d[n].copy_(host[n], non_blocking=True)
@@ -534,7 +565,7 @@ def run_ours(args):
         torch.cuda.synchronize(device)
         barrier(dist, device)
         loc = sum(a.elapsed_time(b) for a, b in zip(e0, e1)) / 1e3
-        js, jb = aggregate(dist, loc, float(step_bytes * Ke), device)
+        js, jb = aggregate(dist, loc, float(wb.step_bytes * Ke), device)
         e2e = {"value": jb / js / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": Ke, "ms_per_step": 1e3 * js / Ke}
 
@@ -542,44 +573,117 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
 
-    del step_graphs, kern_graphs, multi_graph, rem_graph
+    del step_graphs, multi_graph, rem_graph
     if dist is not None:
         dist.barrier(device_ids=[device.index])
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    # ep_layout_dispatch runs as one grid when T <= 128, k <= 8 and a row fits 128 threads
-    units = w.d // 16 if w.quant_mode == 2 else w.d // 8
-    one_grid = w.B > 0 and w.T <= 128 and w.k <= 8 and units <= 1024
-    launches_per_step = 2 if one_grid else 3
     cfg = config_dict(w, args)
-    cfg["l2"] = ("%d buffer sets in rotation: consecutive steps touch disjoint memory "
-                 "(%.0f MB algorithmic per step, L2 126 MB)" % (R, step_bytes / 1e6)) if R > 1 else \
-        cfg["l2"]
+    if R > 1:
+        cfg["l2"] = ("%d buffer sets in rotation: consecutive steps touch disjoint memory "
+                     "(%.0f MB algorithmic per step, L2 126 MB)" % (R, wb.step_bytes / 1e6))
     cfg["timing"] = ("K steps as replays of a CUDA graph of %d consecutive steps (ep_layout_dispatch -> "
                      "ep_combine, programmatic launch edges), CUDA events around the whole timed region; "
                      "step_latency_us_median: single-step graph replays with events around each" % S)
+    lps = wb.launches_per_step
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_s / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": cfg,
         "tokens_per_s": job_tokens / job_s,
-        "bytes_per_step": step_bytes,
+        "bytes_per_step": wb.step_bytes,
         "step_latency_us_median": 1e3 * statistics.median(step_ms),
         "kernels": kernels,
-        "comm_gbs_dispatch": n_routed * w.d * (1 if w.quant_mode == 2 else 2) / (kern_ms["dispatch"] * 1e-3) / 1e9,
+        "layout_then_dispatch_us": 1e3 * kern_ms["layout+dispatch"],
+        "layout_dispatch_one_call_us": 1e3 * kern_ms["layout_dispatch"],
+        "comm_gbs_dispatch": wb.n_routed * w.d * (1 if w.quant_mode == 2 else 2)
+        / (kern_ms["dispatch"] * 1e-3) / 1e9,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clocks.summary(),
-        "gpu_launches": launches_per_step * K,
-        "gpu_launches_latency_loop": launches_per_step * n_lat,
-        "gpu_launches_kernel_loops": (5 + (launches_per_step - 1)) * n_rep * S,
-        "layout_then_dispatch_us": 1e3 * kern_ms["layout+dispatch"],
-        "layout_dispatch_one_call_us": 1e3 * kern_ms["layout_dispatch"],
+        "gpu_launches": lps * K,
+        "gpu_launches_latency_loop": lps * n_lat,
+        "gpu_launches_kernel_loops": (5 + lps) * n_rep * S,
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def fit_latency_bandwidth(points):
+    """Least-squares fit of t = L + V / BW over (V bytes, t seconds) points."""
+    V = np.array([p[0] for p in points], dtype=np.float64)
+    t = np.array([p[1] for p in points], dtype=np.float64)
+    A = np.stack([np.ones_like(V), V], axis=1)
+    (L, inv_bw), *_ = np.linalg.lstsq(A, t, rcond=None)
+    return {"L_us": 1e6 * L, "BW_eff_gbs": (1.0 / inv_bw) / 1e9 if inv_bw > 0 else None}
+
+
+def run_sweep(args, device):
+    """Tokens-per-rank sweep (P = 16, T in 1..4096) and the other named workloads:
+    per-kernel times and GB/s, step time, and a latency/bandwidth fit per kernel.
+    Writes one JSON document to --sweep-out and prints a table."""
+    import torch
+    from combine_ep_layout_12_b200 import workloads as wl
+    names = args.sweep.split(",") if args.sweep != "all" else (
+        ["sweep_T%d_q%d" % (T, q) for q in (2, 0) for T in wl.SWEEP_T] +
+        ["decode", "skewed", "prefill", "tiny_q2"])
+    stream = torch.cuda.Stream(device)
+    peak, _ = measured_peak()
+    results = []
+    for name in names:
+        w = wl.get(name)
+        try:
+            inp = wl.generate(w)
+            wb = Workbench(w, inp, device, stream, args.sets, args.flush_mb)
+        except MemoryError as exc:
+            results.append({"workload": name, "skipped": str(exc)})
+            print("%-18s skipped: %s" % (name, exc), flush=True)
+            continue
+        steps = max(wb.S, min(args.steps, 600))
+        g = wb.steps_graph(wb.S)
+        wb.replay(g, 2)
+        n = max(1, steps // wb.S)
+        step_ms = wb.replay(g, n) / (n * wb.S)
+        if wb.flush is not None:
+            fg = wb.capture(lambda: [wb.flush.zero_() for _ in range(wb.S)])
+            wb.replay(fg, 1)
+            step_ms -= wb.replay(fg, n) / (n * wb.S)
+        kern_ms, _ = wb.kernel_times(steps)
+        for p, _ in wb.sets:
+            assert p.buf.check(stream) == 0
+        rec = {"workload": name, "B": w.B, "T": w.T, "P": w.P, "d": w.d, "E": w.E, "k": w.k,
+               "quant_mode": w.quant_mode, "sets": wb.R, "step_us": 1e3 * step_ms,
+               "step_gbs": wb.step_bytes / (step_ms * 1e-3) / 1e9,
+               "tokens_per_s": w.B / (step_ms * 1e-3), "bytes": wb.kbytes,
+               "layout_dispatch_one_call_us": 1e3 * kern_ms["layout_dispatch"]}
+        for k in ("layout", "dispatch", "combine"):
+            rec[k + "_us"] = 1e3 * kern_ms[k]
+            rec[k + "_gbs"] = wb.kbytes[k] / (kern_ms[k] * 1e-3) / 1e9
+            rec[k + "_frac_of_measured"] = rec[k + "_gbs"] / peak
+        results.append(rec)
+        print("%-18s T=%-5d step %8.1f us %7.0f GB/s | layout %7.1f us | dispatch %8.1f us %6.0f GB/s | "
+              "combine %8.1f us %6.0f GB/s" % (name, w.T, rec["step_us"], rec["step_gbs"], rec["layout_us"],
+                                               rec["dispatch_us"], rec["dispatch_gbs"], rec["combine_us"],
+                                               rec["combine_gbs"]), flush=True)
+        del wb, g
+        torch.cuda.empty_cache()
+    fits = {}
+    for q in (0, 2):
+        pts = [r for r in results if r.get("workload", "").startswith("sweep_") and
+               r.get("quant_mode") == q and "step_us" in r]
+        if len(pts) >= 3:
+            fits["q%d" % q] = {k: fit_latency_bandwidth([(r["bytes"][k], r[k + "_us"] * 1e-6) for r in pts])
+                               for k in ("dispatch", "combine")}
+            fits["q%d" % q]["step"] = fit_latency_bandwidth(
+                [(sum(r["bytes"].values()), r["step_us"] * 1e-6) for r in pts])
+    doc = {"peak_gbs": peak, "results": results, "fits": fits}
+    if args.sweep_out:
+        with open(args.sweep_out, "w") as f:
+            json.dump(doc, f, indent=1)
+    print(json.dumps({"fits": fits}), flush=True)
     return 0
 
 
