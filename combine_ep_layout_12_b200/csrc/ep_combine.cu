@@ -23,6 +23,10 @@ namespace {
 
 enum : int { kSkip = 0, kRouted = 1, kCopy = 2, kConst = 3 };
 
+// Per-rank batches up to this size derive their rows from the routing (the scan of
+// the earlier tokens' ids stays within one load per thread).
+constexpr int kCombineSelfRowsMaxT = 256;
+
 struct CombineArgs {
     const uint16_t* expert_out;  // [rows][d]
     const int32_t* topk_idx;     // [B][k]
@@ -37,6 +41,8 @@ struct CombineArgs {
     long long rows;
     int d, k, E, Z, C, K;
     int chunks;                  // CTAs per token
+    int self_rows;               // derive receive rows from topk_idx instead of reading dst_pos
+    int T, P, M;
 };
 
 __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
@@ -62,14 +68,23 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
     const int v_begin = c * span;
     const int v_end = min(nvec, v_begin + span);
 
-    pdl_wait();
+    // With self_rows the prologue only reads the routing (topk_idx, topk_weights),
+    // which was complete before the preceding kernels started, so it runs before
+    // griddepcontrol.wait and overlaps their tail; the expert outputs are read and
+    // y is written only after the wait.
+    __shared__ int s_rows[KMAX], s_g[KMAX], s_cnt[KMAX];
+    if (a.self_rows) {
+        routing_rows(a.topk_idx, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt);
+    } else {
+        pdl_wait();
+    }
     pdl_launch_dependents();
 
     unsigned bad = 0;
     if (threadIdx.x < a.k) {
         const size_t i = (size_t)t * a.k + threadIdx.x;
         const int g = a.topk_idx[i];
-        const int dp = a.dst_pos[i];
+        const int dp = a.self_rows ? s_rows[threadIdx.x] : a.dst_pos[i];
         int kind = kSkip;
         long long src = 0;
         if (g >= 0 && g < a.E) {
@@ -89,6 +104,7 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
         s_src[threadIdx.x] = src;
         s_w[threadIdx.x] = a.topk_weights[i];
     }
+    if (a.self_rows) pdl_wait();
     if (threadIdx.x < 32) report_err(a.err, bad);
     __syncthreads();
 
@@ -164,6 +180,10 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
     a.Z = s.Z;
     a.C = s.C;
     a.K = s.K;
+    a.T = s.T;
+    a.P = s.P;
+    a.M = s.M;
+    a.self_rows = s.T <= kCombineSelfRowsMaxT ? 1 : 0;
     // One CTA per token when that fills the GPU in about one wave; otherwise split
     // each token's columns over up to nvec / NT CTAs.
     const int nvec = s.d / 8;

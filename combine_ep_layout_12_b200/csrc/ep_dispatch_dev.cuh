@@ -24,45 +24,11 @@ struct DispatchArgs {
     int d, k;
 };
 
-// Receive rows of token t computed from the routing alone (used when T is small):
-// the slot of a routed id g is the number of earlier tokens of the same rank that
-// routed to g (a token counts once), which is exactly the slot the layout kernel
-// assigns.  The earlier tokens' ids come from L2 while the x row load is in
-// flight.  s_g, s_cnt: k-entry shared arrays.  Ends with s_rows published.
-__device__ void compute_rows(const DispatchArgs& a, int t, int* s_rows, int* s_g, int* s_cnt) {
-    const int k = a.k;
-    if (threadIdx.x < k) {
-        const int j = threadIdx.x;
-        const int g = a.topk_idx[(size_t)t * k + j];
-        bool routed = g >= 0 && g < a.E;
-        for (int jj = 0; jj < j; ++jj)
-            if (a.topk_idx[(size_t)t * k + jj] == g) routed = false;  // repeated id: dropped
-        s_g[j] = routed ? g : -1;
-        s_cnt[j] = 0;
-    }
-    __syncthreads();
-    const int r = t / a.T;
-    for (int tt = r * a.T + (int)threadIdx.x; tt < t; tt += blockDim.x) {
-        const int32_t* ids = a.topk_idx + (size_t)tt * k;
-        unsigned hit = 0;
-        for (int jj = 0; jj < k; ++jj) {
-            const int v = __ldg(ids + jj);
-            for (int j = 0; j < k; ++j) {
-                const int g = s_g[j];
-                if (g >= 0 && v == g) hit |= 1u << j;
-            }
-        }
-        while (hit) {
-            const int j = __ffs(hit) - 1;
-            hit &= hit - 1;
-            atomicAdd(&s_cnt[j], 1);
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < k) {
-        const int g = s_g[threadIdx.x];
-        s_rows[threadIdx.x] = g >= 0 ? g * a.P * a.M + r * a.M + s_cnt[threadIdx.x] : -1;
-    }
+// Receive rows of token t computed from the routing alone (used when T is small),
+// while the x row load is in flight.
+__device__ __forceinline__ void compute_rows(const DispatchArgs& a, int t, int* s_rows, int* s_g,
+                                             int* s_cnt) {
+    routing_rows(a.topk_idx, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt);
 }
 
 // Receive rows of token t into shared memory; out-of-range rows are skipped and flagged.

@@ -155,6 +155,49 @@ __device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
     if (all && (int)(threadIdx.x & 31) == __ffs(active) - 1) atomicOr(err_word, all);
 }
 
+// Receive rows of token t derived from the routing alone, for small per-rank
+// batches: the slot of a routed id g is the number of earlier tokens of the same
+// rank that picked g (a token counts once), which is exactly the slot the layout
+// kernels assign; a routed id repeated inside the token gets row -1 after its
+// first occurrence.  The earlier tokens' ids come from L2.  s_rows, s_g, s_cnt:
+// k-entry shared arrays.  All threads of the CTA call it; on return s_rows[j] is
+// written by thread j (j < k) and not yet published to the other threads.
+__device__ inline void routing_rows(const int32_t* topk_idx, int t, int k, int E, int T, int P,
+                                    int M, int* s_rows, int* s_g, int* s_cnt) {
+    if (threadIdx.x < k) {
+        const int j = threadIdx.x;
+        const int g = topk_idx[(size_t)t * k + j];
+        bool routed = g >= 0 && g < E;
+        for (int jj = 0; jj < j; ++jj)
+            if (topk_idx[(size_t)t * k + jj] == g) routed = false;  // repeated id: dropped
+        s_g[j] = routed ? g : -1;
+        s_cnt[j] = 0;
+    }
+    __syncthreads();
+    const int r = t / T;
+    for (int tt = r * T + (int)threadIdx.x; tt < t; tt += blockDim.x) {
+        const int32_t* ids = topk_idx + (size_t)tt * k;
+        unsigned hit = 0;
+        for (int jj = 0; jj < k; ++jj) {
+            const int v = __ldg(ids + jj);
+            for (int j = 0; j < k; ++j) {
+                const int g = s_g[j];
+                if (g >= 0 && v == g) hit |= 1u << j;
+            }
+        }
+        while (hit) {
+            const int j = __ffs(hit) - 1;
+            hit &= hit - 1;
+            atomicAdd(&s_cnt[j], 1);
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < k) {
+        const int g = s_g[threadIdx.x];
+        s_rows[threadIdx.x] = g >= 0 ? g * P * M + r * M + s_cnt[threadIdx.x] : -1;
+    }
+}
+
 }  // namespace ep
 
 #endif  // __CUDACC__
