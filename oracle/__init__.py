@@ -20,7 +20,7 @@ ERR_DUP_ID = 0x2
 
 class OrcCfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
-        "B", "d", "k", "P", "M", "E", "n_zero", "n_copy", "n_const", "quant_mode")]
+        "B", "d", "k", "P", "M", "E", "n_zero", "n_copy", "n_const", "quant_mode", "layout")]
 
 
 _lib = None
@@ -49,6 +49,8 @@ def load(path=None):
     lib.orc_bf16_to_f32.restype = ctypes.c_float
     lib.orc_f32_to_bf16_n.argtypes = [P, P, i64]
     lib.orc_f32_to_bf16_n.restype = None
+    lib.orc_receive_rows.argtypes = [P]
+    lib.orc_receive_rows.restype = i64
     if path == _build.LIB or os.path.abspath(path) == os.path.abspath(_build.LIB):
         _lib, _lib_path = lib, _build.LIB
     return lib
@@ -62,8 +64,17 @@ def _c(a, dtype):
     return None if a is None else np.ascontiguousarray(a, dtype=dtype)
 
 
-def make_cfg(B, d, k, P, M, E, n_zero=0, n_copy=0, n_const=0, quant_mode=0):
-    return OrcCfg(B, d, k, P, M, E, n_zero, n_copy, n_const, quant_mode)
+def make_cfg(B, d, k, P, M, E, n_zero=0, n_copy=0, n_const=0, quant_mode=0, layout=0):
+    """layout 0: low-latency receive rows (E*P*M); 1: packed rows (B*k)."""
+    return OrcCfg(B, d, k, P, M, E, n_zero, n_copy, n_const, quant_mode, layout)
+
+
+def receive_rows(cfg, lib=None):
+    lib = lib or load()
+    n = int(lib.orc_receive_rows(ctypes.byref(cfg)))
+    if n < 0:
+        raise ValueError("oracle rejected the configuration")
+    return n
 
 
 def _check(rc, name):
@@ -73,7 +84,7 @@ def _check(rc, name):
 
 def layout(cfg, topk_idx, lib=None):
     """Returns dict(expert_count, expert_offset, recv_count [E,P], dst_pos [B,k],
-    recv_src [E*P*M], err)."""
+    recv_src [rows], err); rows = E*P*M (low-latency) or B*k (packed)."""
     lib = lib or load()
     E_tot = cfg.E + cfg.n_zero + cfg.n_copy + cfg.n_const
     idx = _c(topk_idx, np.int32)
@@ -82,7 +93,7 @@ def layout(cfg, topk_idx, lib=None):
         expert_offset=np.zeros(E_tot + 1, np.int32),
         recv_count=np.zeros((cfg.E, cfg.P), np.int32),
         dst_pos=np.zeros((cfg.B, cfg.k), np.int32),
-        recv_src=np.zeros(cfg.E * cfg.P * cfg.M, np.int32),
+        recv_src=np.zeros(receive_rows(cfg, lib), np.int32),
     )
     err = np.zeros(1, np.uint32)
     rc = lib.orc_layout(ctypes.byref(cfg), _ptr(idx), _ptr(out["expert_count"]),

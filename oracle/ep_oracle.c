@@ -64,6 +64,7 @@ typedef struct {
     int32_t n_copy;     /* copy experts */
     int32_t n_const;    /* constant experts */
     int32_t quant_mode; /* 0: bf16 pass-through, 2: dynamic int8 */
+    int32_t layout;     /* 0: low-latency rows, 1: packed rows */
 } orc_cfg;
 
 /* ---- bf16 <-> fp32, written from the format definition ------------------- */
@@ -94,10 +95,17 @@ static int cfg_ok(const orc_cfg* c) {
     if (c->P <= 0 || c->M < 0 || c->E <= 0) return 0;
     if (c->n_zero < 0 || c->n_copy < 0 || c->n_const < 0) return 0;
     if (c->B % c->P != 0 || c->E % c->P != 0) return 0;
-    if (c->B / c->P > c->M) return 0;
+    if (c->layout != 0 && c->layout != 1) return 0;
+    if (c->layout == 0 && c->B / c->P > c->M) return 0;
     if (c->quant_mode != 0 && c->quant_mode != 2) return 0;
     return 1;
 }
+
+/* Receive rows the layout addresses: E*P*M (low-latency) or B*k (packed). */
+static int64_t orc_rows(const orc_cfg* c) {
+    return c->layout == 1 ? (int64_t)c->B * c->k : (int64_t)c->E * c->P * c->M;
+}
+int64_t orc_receive_rows(const orc_cfg* c) { return cfg_ok(c) ? orc_rows(c) : -1; }
 
 /* Exported for the tests that pin the format helpers. */
 uint16_t orc_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }
@@ -108,15 +116,20 @@ void orc_f32_to_bf16_n(const float* in, uint16_t* out, int64_t n) {
 
 /*
  * Layout: counts, exclusive prefix, destination row of every routed pick and
- * the source token of every received row, low-latency receive layout
- * recv[g][r*M + slot] with g in [0, E), r the source rank.
+ * the source token of every received row.  slot = the pick's rank among rank
+ * r's tokens that routed to g, in token order.  Receive row:
+ *   low-latency (layout 0): g*P*M + r*M + slot   (a [E][P*M] buffer; the
+ *                           Ascend/DeepEP low-latency form [L][P*M] per rank)
+ *   packed      (layout 1): expert_offset[g] + sum_{r' < r} recv_count[g][r'] + slot
+ *                           (rows contiguous per expert, then per source rank:
+ *                           the dense [A][H] expand_x of the Ascend page)
  *
  * expert_count  [E + Z + C + K]      picks per expert id (routed and special)
  * expert_offset [E + Z + C + K + 1]  exclusive prefix of expert_count
  * recv_count    [E][P]               rows of expert g sent by source rank r
  * dst_pos       [B][k]               global receive row, or -1 if not routed
- * recv_src      [E * P * M]          source token of each received row; -1 in
- *                                    rows nobody wrote
+ * recv_src      [rows]               source token of each received row; -1 in
+ *                                    rows nobody wrote (rows = E*P*M or B*k)
  */
 int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
                int32_t* expert_offset, int32_t* recv_count, int32_t* dst_pos,
@@ -129,9 +142,10 @@ int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
     const int64_t T = c->B / c->P;
     uint32_t err = 0;
 
+    const int64_t rows = orc_rows(c);
     for (int64_t g = 0; g < E_tot; ++g) expert_count[g] = 0;
     for (int64_t i = 0; i < E * P; ++i) recv_count[i] = 0;
-    for (int64_t i = 0; i < E * P * M; ++i) recv_src[i] = -1;
+    for (int64_t i = 0; i < rows; ++i) recv_src[i] = -1;
 
     for (int64_t r = 0; r < P; ++r) {
         for (int64_t t = r * T; t < (r + 1) * T; ++t) {
@@ -157,9 +171,13 @@ int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
                 int64_t slot = recv_count[g * P + r];
                 recv_count[g * P + r] += 1;
                 expert_count[g] += 1;
-                int64_t row = g * P * M + r * M + slot;
-                dst_pos[t * k + j] = (int32_t)row;
-                recv_src[row] = (int32_t)t;
+                if (c->layout == 0) {
+                    int64_t row = g * P * M + r * M + slot;
+                    dst_pos[t * k + j] = (int32_t)row;
+                    recv_src[row] = (int32_t)t;
+                } else {
+                    dst_pos[t * k + j] = (int32_t)slot; /* turned into a row below */
+                }
             }
         }
     }
@@ -170,6 +188,25 @@ int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
         run += expert_count[g];
     }
     expert_offset[E_tot] = (int32_t)run;
+
+    if (c->layout == 1) {
+        /* second pass: rows need every rank's counts of the lower experts */
+        for (int64_t t = 0; t < c->B; ++t) {
+            int64_t r = t / T;
+            for (int64_t j = 0; j < k; ++j) {
+                int64_t g = topk_idx[t * k + j];
+                if (g < 0 || g >= E || dst_pos[t * k + j] < 0) {
+                    dst_pos[t * k + j] = -1;
+                    continue;
+                }
+                int64_t base = expert_offset[g];
+                for (int64_t rr = 0; rr < r; ++rr) base += recv_count[g * P + rr];
+                int64_t row = base + dst_pos[t * k + j];
+                dst_pos[t * k + j] = (int32_t)row;
+                recv_src[row] = (int32_t)t;
+            }
+        }
+    }
     *err_bits = err;
     return ORC_OK;
 }

@@ -78,8 +78,11 @@ def float_to_bf16_bits(f):
     return bits >> 16
 
 
-def layout(topk_idx, B, k, P, M, E, n_special):
-    """Returns (expert_count, recv_count[g][r], dst_pos[t][j], recv_src dict row->t, err)."""
+def layout(topk_idx, B, k, P, M, E, n_special, packed=False):
+    """Returns (expert_count, recv_count[g][r], dst_pos[t][j], recv_src dict row->t, err).
+    packed: rows of expert g come after every pick of a lower expert id, and within
+    g the rows of rank r after those of lower ranks (contiguous per expert, then
+    per rank); otherwise row = g*P*M + r*M + slot."""
     E_tot = E + n_special
     T = B // P
     expert_count = [0] * E_tot
@@ -110,11 +113,25 @@ def layout(topk_idx, B, k, P, M, E, n_special):
                 row_ids = [int(v) for v in topk_idx[t2]]
                 if g in row_ids:
                     slot += 1
-            row = g * P * M + r * M + slot
-            dst_pos[t][j] = row
-            recv_src[row] = t
+            if packed:
+                dst_pos[t][j] = (g, r, slot)  # resolved below, once all counts are known
+            else:
+                row = g * P * M + r * M + slot
+                dst_pos[t][j] = row
+                recv_src[row] = t
             recv_count[g][r] += 1
             expert_count[g] += 1
+    if packed:
+        for t in range(B):
+            for j in range(k):
+                if dst_pos[t][j] == -1:
+                    continue
+                g, r, slot = dst_pos[t][j]
+                lower_experts = sum(expert_count[h] for h in range(g))
+                lower_ranks = sum(recv_count[g][q] for q in range(r))
+                row = lower_experts + lower_ranks + slot
+                dst_pos[t][j] = row
+                recv_src[row] = t
     return expert_count, recv_count, dst_pos, recv_src, err
 
 

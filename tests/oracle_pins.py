@@ -100,7 +100,7 @@ def pin_bf16_format(lib):
 # ----------------------------------------------------------------------------- layout
 
 
-def _compare_layout(name, out, ref, B, k, P, M, E):
+def _compare_layout(name, out, ref, B, k, P, M, E, rows=None):
     fails = []
     ec, rc, dp, rs, err = ref
     if list(out["expert_count"]) != list(ec):
@@ -114,7 +114,7 @@ def _compare_layout(name, out, ref, B, k, P, M, E):
         fails.append("%s: recv_count differs from brute force" % name)
     if out["dst_pos"].tolist() != dp:
         fails.append("%s: dst_pos differs from brute force" % name)
-    want_src = np.full(E * P * M, -1, np.int64)
+    want_src = np.full(E * P * M if rows is None else rows, -1, np.int64)
     for row, t in rs.items():
         want_src[row] = t
     if not np.array_equal(out["recv_src"].astype(np.int64), want_src):
@@ -194,6 +194,90 @@ def pin_layout_random_brute(lib):
         fails.append("bad/duplicate ids: error bits %#x" % out["err"])
     if out["dst_pos"][0].tolist() != [0 * 3 + 0, -1, 1 * 3 + 0]:
         fails.append("duplicate id: first occurrence must be routed, the second dropped")
+    return fails
+
+
+def pin_layout_packed_brute(lib):
+    """Packed rows against the brute force's definition (rows after every pick of a
+    lower expert, then after the lower ranks' rows of the same expert)."""
+    fails = []
+    rng = np.random.default_rng(15)
+    for trial in range(10):
+        P = int(rng.integers(1, 4))
+        T = int(rng.integers(1, 7))
+        B = P * T
+        L = int(rng.integers(1, 4))
+        E = L * P
+        Z, C, K = (int(v) for v in rng.integers(0, 2, 3))
+        k = int(rng.integers(1, 6))
+        E_tot = E + Z + C + K
+        if trial % 3 == 0:
+            idx = rng.integers(-2, E_tot + 2, size=(B, k)).astype(np.int32)
+        else:
+            idx = np.stack([np.concatenate([rng.permutation(E_tot), -np.ones(max(0, k - E_tot), int)])[:k]
+                            for _ in range(B)]).astype(np.int32)
+        cfg = oracle.make_cfg(B, 16, k, P, 0, E, Z, C, K, 0, layout=1)
+        out = oracle.layout(cfg, idx, lib=lib)
+        ref = brute.layout(idx.tolist(), B, k, P, 0, E, Z + C + K, packed=True)
+        fails += _compare_layout("packed trial %d" % trial, out, ref, B, k, P, 0, E, rows=B * k)
+    for fx in ("ascend_topk_single_operator.txt", "ascend_topk_graph_mode.txt"):
+        mat, meta = read_topk_fixture(fx)
+        E, k = meta["E"], meta["k"]
+        for P in (1, 16):
+            idx = np.tile(mat, (P, 1))
+            B = idx.shape[0]
+            cfg = oracle.make_cfg(B, 16, k, P, 0, E, meta["n_zero"], meta["n_copy"], 0, 0, layout=1)
+            out = oracle.layout(cfg, idx, lib=lib)
+            ref = brute.layout(idx.tolist(), B, k, P, 0, E, meta["n_zero"] + meta["n_copy"], packed=True)
+            fails += _compare_layout("%s packed P=%d" % (fx, P), out, ref, B, k, P, 0, E, rows=B * k)
+    return fails
+
+
+def packed_invariant_failures(packed, ll, idx, B, k, P, M, E, name=""):
+    """Properties of the packed rows, and their relation to the low-latency rows of
+    the same routing."""
+    fails = []
+    T, L = B // P, E // P
+    ec, eo, rc = packed["expert_count"], packed["expert_offset"], packed["recv_count"]
+    dp, rs = packed["dst_pos"], packed["recv_src"]
+    for name_, arr in (("expert_count", "expert_count"), ("expert_offset", "expert_offset"),
+                       ("recv_count", "recv_count")):
+        if not np.array_equal(packed[arr], ll[arr]):
+            fails.append("%s: %s differs between the layouts" % (name, name_))
+    ok = dp >= 0
+    if not np.array_equal(ok, ll["dst_pos"] >= 0):
+        fails.append("%s: routed picks differ between the layouts" % name)
+    rows = dp[ok]
+    if np.unique(rows).size != rows.size or (rows.size and rows.max() >= eo[E]):
+        fails.append("%s: packed rows not a permutation of [0, routed picks)" % name)
+    tt = np.repeat(np.arange(B), k).reshape(B, k)
+    if not np.array_equal(rs[dp[ok]], tt[ok]):
+        fails.append("%s: recv_src[dst_pos[t,j]] != t" % name)
+    g = idx[ok]
+    r = tt[ok] // T
+    base = eo[g] + np.array([rc[gg, :rr].sum() for gg, rr in zip(g, r)], dtype=np.int64)
+    ll_slot = ll["dst_pos"][ok] - (g * P * M + r * M)
+    if not np.array_equal(rows - base, ll_slot):
+        fails.append("%s: packed row - run base differs from the low-latency slot" % name)
+    for q in range(P):
+        lo, hi = eo[q * L], eo[(q + 1) * L]
+        mine = (g // L) == q
+        if rows[mine].size and (rows[mine].min() < lo or rows[mine].max() >= hi):
+            fails.append("%s: rank %d's rows are not contiguous" % (name, q))
+            break
+    return fails
+
+
+def pin_layout_packed_invariants(lib):
+    from combine_ep_layout_12_b200 import workloads as wl
+    fails = []
+    for name in ("decode", "skewed"):
+        w = wl.get(name)
+        idx = wl.generate(w, with_x=False)["topk_idx"]
+        args = (w.B, w.d, w.k, w.P, w.M, w.E, w.n_zero, w.n_copy, w.n_const, w.quant_mode)
+        ll = oracle.layout(oracle.make_cfg(*args, layout=0), idx, lib=lib)
+        pk = oracle.layout(oracle.make_cfg(*args, layout=1), idx, lib=lib)
+        fails += packed_invariant_failures(pk, ll, idx, w.B, w.k, w.P, w.M, w.E, name=name)
     return fails
 
 
@@ -549,6 +633,8 @@ ALL_PINS = [
     pin_layout_golden,
     pin_layout_random_brute,
     pin_layout_invariants,
+    pin_layout_packed_brute,
+    pin_layout_packed_invariants,
     pin_mask_experiment,
     pin_quant_brute,
     pin_quant_properties,

@@ -51,6 +51,10 @@ MUTANTS = [
      "for (int64_t j = 0; j < k - 1; ++j) {\n                int64_t g = topk_idx[t * k + j];\n                float w"),
     ("scatter_scale_dropped", "if (c->quant_mode == 2) recv_scale[row] = token_scale[t];",
      "(void)recv_scale;"),
+    ("packed_rank_prefix_dropped", "for (int64_t rr = 0; rr < r; ++rr) base += recv_count[g * P + rr];",
+     "for (int64_t rr = 0; rr < 0; ++rr) base += recv_count[g * P + rr];"),
+    ("packed_rank_prefix_inclusive", "for (int64_t rr = 0; rr < r; ++rr) base += recv_count[g * P + rr];",
+     "for (int64_t rr = 0; rr < r && rr < P - 1; ++rr) base += recv_count[g * P + rr + (r > 1)];"),
 ]
 
 RUNNER = r"""
