@@ -50,14 +50,16 @@ class EPBuffer:
     cfg: an ep_config (see make_config) or any object with the config fields
     (B, d, k, P, M, E, n_zero, n_copy, n_const, quant_mode[, smooth_rows]).
     Views: expert_count [E_tot], expert_offset [E_tot+1], recv_count [E, P],
-    dst_pos [B, k], recv_src [E*P*M], recv_x [E*P*M, d] (int8 or bf16),
-    recv_scale [E*P*M], token_scale [B].
+    dst_pos [B, k], recv_src [rows], recv_x [rows, d] (int8 or bf16),
+    recv_scale [rows], token_scale [B]; rows = E*P*M (low-latency layout) or
+    B*k (packed layout).
     """
 
     def __init__(self, cfg, device=None):
         if not isinstance(cfg, abi.ep_config):
             cfg = make_config(cfg.B, cfg.d, cfg.k, cfg.P, cfg.M, cfg.E, cfg.n_zero, cfg.n_copy,
-                              cfg.n_const, cfg.quant_mode, getattr(cfg, "smooth_rows", 1), 0)
+                              cfg.n_const, cfg.quant_mode, getattr(cfg, "smooth_rows", 1),
+                              getattr(cfg, "layout", 0))
         self.cfg = cfg
         dev = torch.device("cuda" if device is None else device)
         if dev.type != "cuda":
@@ -67,7 +69,7 @@ class EPBuffer:
         self.sizes = {n: int(getattr(sizes, n)) for n in abi.BUFFER_FIELDS}
         c = cfg
         self.E_tot = c.E + c.n_zero + c.n_copy + c.n_const
-        self.rows = c.E * c.P * c.M
+        self.rows = c.B * c.k if c.layout == 1 else c.E * c.P * c.M
         dev = self.device
         self.expert_count = torch.empty(self.E_tot, dtype=torch.int32, device=dev)
         self.expert_offset = torch.empty(self.E_tot + 1, dtype=torch.int32, device=dev)

@@ -183,7 +183,7 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
     a.T = s.T;
     a.P = s.P;
     a.M = s.M;
-    a.self_rows = s.T <= kCombineSelfRowsMaxT ? 1 : 0;
+    a.self_rows = (s.layout == 0 && s.T <= kCombineSelfRowsMaxT) ? 1 : 0;
     // One CTA per token when that fills the GPU in about one wave; otherwise split
     // each token's columns over up to nvec / NT CTAs.
     const int nvec = s.d / 8;

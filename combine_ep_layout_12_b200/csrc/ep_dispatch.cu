@@ -48,7 +48,7 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
     DispatchArgs a = make_dispatch_args(s, p, x, smooth, topk_idx);
     // Small batches per rank: each CTA derives its rows from the routing itself
     // (at most kSelfRowsMaxT earlier tokens to scan), so dispatch overlaps layout.
-    a.self_rows = (topk_idx != nullptr && s.T <= kSelfRowsMaxT) ? 1 : 0;
+    a.self_rows = (topk_idx != nullptr && s.layout == 0 && s.T <= kSelfRowsMaxT) ? 1 : 0;
     int U = 0, NT = 0;
     cudaError_t e = cudaSuccess;
     const dim3 grid(s.B);

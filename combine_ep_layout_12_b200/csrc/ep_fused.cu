@@ -47,7 +47,8 @@ int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_
     const int cpr = (s.T + 31) / 32;
     int U = 0, NT = 0;
     const int units = s.quant_mode == 2 ? s.d / 16 : s.d / 8;
-    const bool fits = s.B > 0 && cpr <= 4 && s.k <= 8 && pick_units(units, 8, &U, &NT) == EP_OK &&
+    const bool fits = s.B > 0 && s.layout == 0 && cpr <= 4 && s.k <= 8 &&
+                      pick_units(units, 8, &U, &NT) == EP_OK &&
                       NT <= 128 && U <= 8;
     if (!fits) {
         const int st = launch_layout(s, p, topk_idx, stream);

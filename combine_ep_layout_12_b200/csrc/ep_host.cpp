@@ -30,24 +30,29 @@ int check_config(const ep_config* c) {
     if (c->B % c->P != 0 || c->E % c->P != 0) return EP_ERR_INVALID_ARG;
     if (c->quant_mode != 0 && c->quant_mode != 2) return EP_ERR_INVALID_ARG;
     if (c->smooth_rows != 0 && c->smooth_rows != 1) return EP_ERR_INVALID_ARG;
-    if (c->layout != 0) return EP_ERR_UNSUPPORTED;
+    if (c->layout != 0 && c->layout != 1) return EP_ERR_UNSUPPORTED;
     if (c->d % 16 != 0) return EP_ERR_INVALID_ARG;
     if (c->k > ep::kMaxK) return EP_ERR_INVALID_ARG;
     if (c->d > ep::kMaxD) return EP_ERR_UNSUPPORTED;
     if (c->E > ep::kMaxE) return EP_ERR_UNSUPPORTED;
     const long long n_special = (long long)c->n_zero + c->n_copy + c->n_const;
     if (n_special > ep::kMaxSpecial) return EP_ERR_UNSUPPORTED;
-    if (c->B / c->P > c->M) return EP_ERR_CAPACITY;
-    const long long rows = (long long)c->E * c->P * c->M;
-    if (rows >= (1LL << 31)) return EP_ERR_CAPACITY;
     if ((long long)c->B * c->k >= (1LL << 31)) return EP_ERR_CAPACITY;
+    if (c->layout == 0) {
+        if (c->B / c->P > c->M) return EP_ERR_CAPACITY;
+        if ((long long)c->E * c->P * c->M >= (1LL << 31)) return EP_ERR_CAPACITY;
+    } else {
+        // packed rows are derived from low-latency-form rows with stride T
+        if ((long long)c->E * c->B >= (1LL << 31)) return EP_ERR_CAPACITY;
+        if ((long long)c->E * c->P > ep::kMaxPackedEP) return EP_ERR_UNSUPPORTED;
+    }
     return EP_OK;
 }
 
 void fill_sizes(const ep_config* c, ep_buffer_sizes* s) {
     const size_t E_tot = (size_t)c->E + c->n_zero + c->n_copy + c->n_const;
     const size_t n_special = (size_t)c->n_zero + c->n_copy + c->n_const;
-    const size_t rows = (size_t)c->E * c->P * c->M;
+    const size_t rows = (size_t)ep::make_shape(*c).rows;
     const size_t esz = c->quant_mode == 2 ? 1 : 2;
     s->expert_count = 4 * E_tot;
     s->expert_offset = 4 * (E_tot + 1);

@@ -23,10 +23,13 @@ constexpr int kMaxSpecial = 2048;  // zero + copy + const experts
 constexpr int kMaxK = 16;          // picks per token (Ascend: 0 < K <= 16)
 constexpr int kMaxD = 32768;     // 256 threads x 8 units of 16 elements
 
+constexpr int kMaxPackedEP = 24576;  // E * P of the packed layout (the pack kernel's shared table)
+
 struct Shape {
     int B, d, k, P, M, E, Z, C, K, T, L, E_tot, n_special;
     int quant_mode;
-    long long rows;  // E * P * M receive rows
+    int layout;      // 0 low-latency, 1 packed
+    long long rows;  // receive rows: E * P * M (low-latency) or B * k (packed)
 };
 
 inline Shape make_shape(const ep_config& c) {
@@ -38,7 +41,8 @@ inline Shape make_shape(const ep_config& c) {
     s.n_special = c.n_zero + c.n_copy + c.n_const;
     s.E_tot = c.E + s.n_special;
     s.quant_mode = c.quant_mode;
-    s.rows = (long long)c.E * c.P * c.M;
+    s.layout = c.layout;
+    s.rows = c.layout == 1 ? (long long)c.B * c.k : (long long)c.E * c.P * c.M;
     return s;
 }
 

@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
                     const int g = ids[j];
                     const int slot = my_pre[g] + __popc(my_mask[g] & lt);
                     row = g * a.P * a.M + r * a.M + slot;
-                    a.recv_src[row] = t;
+                    if (a.recv_src) a.recv_src[row] = t;
                 }
                 a.dst_pos[(size_t)t * k + j] = row;
             }
@@ -174,10 +174,73 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
     if (threadIdx.x == 0) a.ws->done = 0u;  // re-arm the ticket for the next launch
 }
 
+// Packed layout, second step: the layout kernels left each routed pick's row in
+// low-latency form with stride T (g*P*T + r*T + slot); with every rank's counts
+// known, the row becomes expert_offset[g] + sum_{r' < r} recv_count[g][r'] + slot,
+// and recv_src is written at it.  Each CTA builds the (expert, rank) base table in
+// shared memory, then converts a grid-strided share of the picks.
+__global__ void __launch_bounds__(256) layout_pack_kernel(const int32_t* expert_offset,
+                                                          const int32_t* recv_count, int32_t* dst_pos,
+                                                          int32_t* recv_src, int B, int k, int P,
+                                                          int T, int E) {
+    extern __shared__ int base[];  // [E][P]
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int g = threadIdx.x; g < E; g += blockDim.x) {
+        int run = expert_offset[g];
+        for (int r = 0; r < P; ++r) {
+            base[g * P + r] = run;
+            run += recv_count[g * P + r];
+        }
+    }
+    __syncthreads();
+    const long long n = (long long)B * k;
+    const int PT = P * T;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int v = dst_pos[i];
+        if (v < 0) continue;
+        const int g = v / PT;
+        const int rem = v - g * PT;
+        const int r = rem / T;
+        const int row = base[g * P + r] + (rem - r * T);
+        dst_pos[i] = row;
+        recv_src[row] = (int)(i / k);
+    }
+}
+
 }  // namespace
 
 int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
                   cudaStream_t stream) {
+    if (s.layout == 1 && s.B > 0) {
+        // counts and low-latency-form rows (stride T, no recv_src), then pack
+        Shape ll = s;
+        ll.layout = 0;
+        ll.M = s.T;
+        ll.rows = (long long)s.E * s.P * s.T;
+        ep_buffer_ptrs q = p;
+        q.recv_src = nullptr;
+        const int st = launch_layout(ll, q, topk_idx, stream);
+        if (st != EP_OK) return st;
+        const size_t smem = sizeof(int) * (size_t)s.E * s.P;
+        static bool attr_pack[64] = {false};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 64 && !attr_pack[dev]) {
+            if (cudaFuncSetAttribute(layout_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(sizeof(int) * kMaxPackedEP)) != cudaSuccess)
+                return EP_ERR_CUDA;
+            attr_pack[dev] = true;
+        }
+        long long grid = ((long long)s.B * s.k + 1023) / 1024;
+        if (grid > (long long)num_sms() * 4) grid = (long long)num_sms() * 4;
+        if (grid < 1) grid = 1;
+        cudaError_t e = launch_pdl(layout_pack_kernel, dim3((unsigned)grid), dim3(256), smem, stream,
+                                   (const int32_t*)p.expert_offset, (const int32_t*)p.recv_count,
+                                   p.dst_pos, p.recv_src, s.B, s.k, s.P, s.T, s.E);
+        return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    }
     if (s.B == 0) {
         // no tokens: counts are all zero
         cudaError_t e1 = cudaMemsetAsync(p.expert_count, 0, sizeof(int32_t) * s.E_tot, stream);

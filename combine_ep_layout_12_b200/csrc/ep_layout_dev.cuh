@@ -201,7 +201,7 @@ __device__ __forceinline__ void layout_small_body(const LayoutArgs& a, int cpr, 
                 int before = 0;  // the rank's tokens in its earlier chunks that routed to g
                 for (int cc = 0; cc < c; ++cc) before += __popc(rank_masks[(size_t)cc * E + g]);
                 row = g * P * a.M + r * a.M + before + __popc(my_mask[g] & lt);
-                a.recv_src[row] = t;
+                if (a.recv_src) a.recv_src[row] = t;
             }
             a.dst_pos[(size_t)t * k + j] = row;
         }

@@ -39,6 +39,7 @@ class Workload:
     zipf_s: float = 1.2
     smooth: str = "none"
     seed: int = 0
+    layout: int = 0  # 0: low-latency receive rows [E][P*M]; 1: packed rows [B*k]
 
     @property
     def T(self):
@@ -54,8 +55,8 @@ class Workload:
 
     @property
     def rows(self):
-        """Receive rows of the low-latency layout over all logical ranks: E * P * M."""
-        return self.E * self.P * self.M
+        """Receive rows: E * P * M (low-latency layout) or B * k (packed layout)."""
+        return self.B * self.k if self.layout == 1 else self.E * self.P * self.M
 
     def with_(self, **kw):
         return replace(self, **kw)
@@ -86,6 +87,12 @@ SWEEP_T = (1, 4, 16, 64, 256, 1024, 4096)
 for _T in SWEEP_T:
     for _qm in (0, 2):
         WORKLOADS[f"sweep_T{_T}_q{_qm}"] = _sweep(_T, _qm)
+# the same workloads with the packed receive layout (rows contiguous per expert,
+# no per-(expert, rank) padding)
+for _name in list(WORKLOADS):
+    if not _name.startswith("tiny_q0"):
+        WORKLOADS[_name + "_packed"] = replace(WORKLOADS[_name], name=_name + "_packed", layout=1)
+WORKLOADS["tiny_q0_packed"] = replace(WORKLOADS["tiny_q0"], name="tiny_q0_packed", layout=1)
 
 
 def get(name):

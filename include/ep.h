@@ -16,11 +16,14 @@
  *
  *   ep_layout   counts per expert and per (expert, source rank), their exclusive
  *               prefix, the receive row of every routed pick and the source token
- *               of every receive row.  Receive layout is the low-latency one:
+ *               of every receive row.  Low-latency receive layout (layout 0):
  *               row = g * P * M + r * M + slot, i.e. a [E][P*M][d] buffer that
- *               rank q reads as [L][P*M][d] starting at expert q*L.  slot is the
- *               rank of token t among rank r's tokens that routed to g, ascending
- *               t (the page states the computation is deterministic).
+ *               rank q reads as [L][P*M][d] starting at expert q*L.  Packed
+ *               layout (layout 1): rows contiguous per expert, then per source
+ *               rank, with no padding (the dense expand_x [A][H] of the Ascend
+ *               page).  slot is the rank of token t among rank r's tokens that
+ *               routed to g, ascending t (the page states the computation is
+ *               deterministic).
  *   ep_dispatch quant_mode 0: expand_x row = x[t] (bf16 bits copied).
  *               quant_mode 2: xf = fp32(x) * smooth_scale, s = 127 / max|xf| over
  *               the row, q = CastToInt8(xf * s) (round half to even, saturate),
@@ -91,7 +94,9 @@ typedef struct CUstream_st* ep_stream_t;
  *   local_expert_num * ep_world_size <= 2048), 1 <= k <= 16 (Constraints:
  *   0 < K <= 16), T = B / P <= M, Z, C, K >= 0 with Z + C + K <= 2048,
  *   E*P*M < 2^31 (int32 row ids), 16 <= d <= 32768 with d % 16 == 0,
- *   quant_mode in {0, 2}, smooth_rows in {0, 1}, layout == 0.
+ *   quant_mode in {0, 2}, smooth_rows in {0, 1}, layout in {0, 1}.  The T <= M
+ *   and E*P*M bounds apply to layout 0; layout 1 needs E*B < 2^31 and
+ *   E*P <= 24576.
  */
 typedef struct {
     int32_t B;           /* tokens over all logical ranks */
@@ -105,7 +110,13 @@ typedef struct {
     int32_t n_const;     /* constant experts (next K ids) */
     int32_t quant_mode;  /* 0: bf16 pass-through; 2: dynamic per-token int8 */
     int32_t smooth_rows; /* 0: no smooth scale; 1: one fp32 [d] vector may be given */
-    int32_t layout;      /* 0: low-latency [E][P*M][d] receive layout */
+    int32_t layout;      /* 0: low-latency [E][P*M][d] receive layout;
+                            1: packed [B*k][d]: the rows of expert g start at
+                               expert_offset[g], those of source rank r after the
+                               lower ranks' (expert_offset[g] + sum_{r'<r}
+                               recv_count[g][r'] + slot); rank q reads rows
+                               [expert_offset[q*L], expert_offset[(q+1)*L]).
+                               M is not used. */
 } ep_config;
 
 /* Byte sizes of the caller-allocated device arrays (0 = not needed). */
@@ -115,11 +126,12 @@ typedef struct {
     size_t recv_count;    /* int32 [E][P]       rows of expert g from source rank r
                              (per receiving rank q: [L][P] = ep_recv_counts) */
     size_t dst_pos;       /* int32 [B][k]       receive row of each pick, -1 if none */
-    size_t recv_src;      /* int32 [E*P*M]      source token of each receive row
+    size_t recv_src;      /* int32 [rows]       source token of each receive row
                              (the combine's source map); rows past a run's count
-                             are not written */
-    size_t recv_x;        /* [E*P*M][d] int8 (quant_mode 2) or bf16 (quant_mode 0) */
-    size_t recv_scale;    /* fp32 [E*P*M]       1/s of the row's token (quant_mode 2) */
+                             are not written.  rows = E*P*M (layout 0) or B*k
+                             (layout 1; rows past expert_offset[E] unused) */
+    size_t recv_x;        /* [rows][d] int8 (quant_mode 2) or bf16 (quant_mode 0) */
+    size_t recv_scale;    /* fp32 [rows]        1/s of the row's token (quant_mode 2) */
     size_t token_scale;   /* fp32 [B]           1/s per token (quant_mode 2) */
     size_t workspace;     /* scratch words; zero-filled by ep_buffer_create */
 } ep_buffer_sizes;

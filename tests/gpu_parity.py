@@ -16,10 +16,10 @@ from combine_ep_layout_12_b200 import workloads as wl
 COMBINE_REL_TOL = 8e-3
 
 
-def ocfg(w, B=None, P=None, M=None):
+def ocfg(w, B=None, P=None, M=None, layout=None):
     return oracle.make_cfg(w.B if B is None else B, w.d, w.k, w.P if P is None else P,
                            w.M if M is None else M, w.E, w.n_zero, w.n_copy, w.n_const,
-                           w.quant_mode)
+                           w.quant_mode, layout=w.layout if layout is None else layout)
 
 
 def bf16_to_f32(bits):
@@ -110,7 +110,7 @@ def check_combine(rep, w, pipe, inp, dev_inp, ref_lay, tokens=None, seed_offset=
         torch.cuda.synchronize()
         pipe.combine(dev_inp)
     y_gpu = runner.bf16_bits(pipe.y[torch.from_numpy(tokens).to(pipe.device)])
-    sub = ocfg(w, B=len(tokens), P=1, M=max(len(tokens), 1))
+    sub = ocfg(w, B=len(tokens), P=1, M=max(len(tokens), 1), layout=0)
     idx = inp["topk_idx"][tokens]
     wts = inp["topk_weights"][tokens]
     x = inp["x"][tokens]

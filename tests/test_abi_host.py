@@ -85,7 +85,8 @@ def test_sizes_bf16_specials():
     (dict(M=2**20), abi.EP_ERR_CAPACITY),           # E*P*M >= 2^31
     (dict(n_zero=-1), abi.EP_ERR_INVALID_ARG),
     (dict(n_const=4096), abi.EP_ERR_UNSUPPORTED),
-    (dict(layout=1), abi.EP_ERR_UNSUPPORTED),
+    (dict(layout=2), abi.EP_ERR_UNSUPPORTED),
+    (dict(layout=1, E=2048, P=16, B=1024, M=64), abi.EP_ERR_UNSUPPORTED),   # E*P above the pack table
     (dict(smooth_rows=2), abi.EP_ERR_INVALID_ARG),
     (dict(P=0), abi.EP_ERR_INVALID_ARG),
 ])
@@ -93,6 +94,14 @@ def test_bad_configs(kw, status):
     with pytest.raises(abi.EPError) as ei:
         abi.ep_buffer_size(cfg(**kw))
     assert ei.value.status == status
+
+
+def test_sizes_packed():
+    s = abi.ep_buffer_size(cfg(layout=1, M=0))       # M is not used by the packed layout
+    rows = 1024 * 8
+    assert s.recv_x == rows * 7168 and s.recv_src == 4 * rows and s.recv_scale == 4 * rows
+    s0 = abi.ep_buffer_size(cfg(layout=1, quant_mode=0, M=0))
+    assert s0.recv_x == rows * 7168 * 2 and s0.recv_scale == 0
 
 
 def test_edge_configs_accepted():

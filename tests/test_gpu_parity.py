@@ -164,6 +164,50 @@ def test_prefill(dev):
     rep.assert_ok()
 
 
+# ----------------------------------------------------------------------------- packed layout
+
+
+@pytest.mark.parametrize("name", ["tiny_q0_packed", "tiny_q2_packed", "decode_packed", "skewed_packed",
+                                  "sweep_T1_q2_packed", "sweep_T16_q2_packed", "sweep_T256_q0_packed"])
+def test_packed(dev, name):
+    """Packed receive rows (contiguous per expert, then per source rank)."""
+    full_check(wl.get(name), dev)
+
+
+@pytest.mark.parametrize("name", ["prefill_packed", "sweep_T4096_q0_packed", "sweep_T4096_q2_packed"])
+def test_packed_large_sampled(dev, name):
+    """The largest configurations in the packed layout (3.8-11 GB instead of
+    120-360 GB low-latency buffers): layout in full, payload on sampled picks,
+    combine on sampled tokens."""
+    w = wl.get(name)
+    rng = np.random.default_rng(4096)
+    tokens = np.sort(rng.choice(w.B, 512, replace=False))
+    full_check(w, dev, tokens=tokens, sample_picks=16384, separate=(w.quant_mode == 2))
+
+
+def test_packed_dirty(dev):
+    w = wl.Workload("ragged_packed", B=111, d=272, k=3, P=3, M=0, E=9, n_zero=1, n_copy=1, n_const=1,
+                    quant_mode=2, smooth="rand", seed=8, layout=1)
+    inp = wl.generate(w)
+    rng = np.random.default_rng(8)
+    idx = np.stack([rng.permutation(w.E_tot)[:w.k] for _ in range(w.B)]).astype(np.int32)
+    idx[1, 2] = -1
+    idx[4, 0] = w.E_tot + 1
+    idx[9] = [2, 2, 5]
+    inp["topk_idx"] = idx
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev, alias_expert_out=False)
+    pipe.layout_dispatch(dev_inp)
+    err = pipe.buf.check()
+    ref = oracle.layout(gp.ocfg(w), idx)
+    assert err == ref["err"] == (oracle.ERR_BAD_ID | oracle.ERR_DUP_ID)
+    rep = gp.Report()
+    gp.check_layout(rep, w, pipe, ref)
+    gp.check_dispatch(rep, w, pipe, inp, ref)
+    gp.check_combine(rep, w, pipe, inp, dev_inp, ref)
+    rep.assert_ok()
+
+
 # ----------------------------------------------------------------------------- fused call
 
 

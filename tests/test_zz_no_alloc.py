@@ -42,7 +42,7 @@ def _outputs(w, dev):
 
 def _cfg(w):
     return abi.make_config(w.B, w.d, w.k, w.P, w.M, w.E, w.n_zero, w.n_copy, w.n_const,
-                           w.quant_mode, 1, 0)
+                           w.quant_mode, 1, w.layout)
 
 
 def _static_layout(w, topk_idx, out, stream):
@@ -60,7 +60,7 @@ def _dirty(w):
     return idx
 
 
-@pytest.mark.parametrize("name", ["decode", "skewed", "dirty"])
+@pytest.mark.parametrize("name", ["decode", "skewed", "dirty", "decode_packed"])
 def test_static_scratch_layout_matches_ep_layout(dev, name):
     if name == "dirty":
         w = wl.get("skewed").with_(name="dirty", n_zero=2, n_copy=1, n_const=3, k=5)
