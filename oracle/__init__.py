@@ -51,6 +51,8 @@ def load(path=None):
     lib.orc_f32_to_bf16_n.restype = None
     lib.orc_receive_rows.argtypes = [P]
     lib.orc_receive_rows.restype = i64
+    lib.orc_dispatch_expert_smooth.argtypes = [P, P, P, P, P, P, P, i64]
+    lib.orc_dispatch_expert_smooth.restype = ctypes.c_int
     if path == _build.LIB or os.path.abspath(path) == os.path.abspath(_build.LIB):
         _lib, _lib_path = lib, _build.LIB
     return lib
@@ -132,6 +134,21 @@ def dispatch(cfg, quant_out, token_scale, dst_pos, rows, lib=None):
     rc = lib.orc_dispatch(ctypes.byref(cfg), _ptr(q), _ptr(ts), _ptr(dp), _ptr(recv_x),
                           _ptr(recv_scale), rows)
     _check(rc, "dispatch")
+    return recv_x, recv_scale
+
+
+def dispatch_expert_smooth(cfg, x_bits, smooth_E, topk_idx, dst_pos, rows, lib=None):
+    """Per-copy quantization with a [E, d] smooth scale, scattered to `rows` receive
+    rows.  Returns (recv_x int8 [rows, d], recv_scale float32 [rows]); rows no pick
+    maps to stay zero."""
+    lib = lib or load()
+    recv_x = np.zeros((rows, cfg.d), np.int8)
+    recv_scale = np.zeros(rows, np.float32)
+    rc = lib.orc_dispatch_expert_smooth(ctypes.byref(cfg), _ptr(_c(x_bits, np.uint16)),
+                                        _ptr(_c(smooth_E, np.float32)), _ptr(_c(topk_idx, np.int32)),
+                                        _ptr(_c(dst_pos, np.int32)), _ptr(recv_x), _ptr(recv_scale),
+                                        rows)
+    _check(rc, "dispatch_expert_smooth")
     return recv_x, recv_scale
 
 

@@ -218,6 +218,31 @@ int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
  *                q = CastToInt8(x_fp32 * s), token_scale = 1 / s.
  * smooth is a [d] fp32 vector or NULL (NULL means no multiply at all).
  */
+/* One row: x_fp32 = fp32(x) (* smooth), s = 127 / max|x_fp32|, q = CastToInt8(x_fp32 * s).
+ * Returns 1 / s, or 0 with q = 0 when amax == 0 or s is not finite.  xf: d floats scratch. */
+static float quantize_row(const uint16_t* x, const float* smooth, int64_t d, float* xf, int8_t* q) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < d; ++i) {
+        float v = bf16_to_f32(x[i]);
+        if (smooth) v = v * smooth[i];
+        xf[i] = v;
+        float a = fabsf(v);
+        if (a > amax) amax = a;
+    }
+    float s = 127.0f / amax;
+    if (amax == 0.0f || !isfinite(s)) {
+        for (int64_t i = 0; i < d; ++i) q[i] = 0;
+        return 0.0f;
+    }
+    for (int64_t i = 0; i < d; ++i) {
+        float y = nearbyintf(xf[i] * s);  /* default rounding: nearest, ties to even */
+        if (y > 127.0f) y = 127.0f;
+        if (y < -128.0f) y = -128.0f;
+        q[i] = (int8_t)y;
+    }
+    return 1.0f / s;
+}
+
 int orc_quantize(const orc_cfg* c, const uint16_t* x, const float* smooth, void* quant_out,
                  float* token_scale) {
     if (!cfg_ok(c) || !x || !quant_out) return ORC_BAD_ARG;
@@ -231,29 +256,7 @@ int orc_quantize(const orc_cfg* c, const uint16_t* x, const float* smooth, void*
     int8_t* q = (int8_t*)quant_out;
     float* xf = (float*)malloc(sizeof(float) * (size_t)d);
     if (!xf) return ORC_BAD_ARG;
-    for (int64_t t = 0; t < B; ++t) {
-        float amax = 0.0f;
-        for (int64_t i = 0; i < d; ++i) {
-            float v = bf16_to_f32(x[t * d + i]);
-            if (smooth) v = v * smooth[i];
-            xf[i] = v;
-            float a = fabsf(v);
-            if (a > amax) amax = a;
-        }
-        float s = 127.0f / amax;
-        if (amax == 0.0f || !isfinite(s)) {
-            for (int64_t i = 0; i < d; ++i) q[t * d + i] = 0;
-            token_scale[t] = 0.0f;
-            continue;
-        }
-        for (int64_t i = 0; i < d; ++i) {
-            float y = nearbyintf(xf[i] * s);  /* default rounding: nearest, ties to even */
-            if (y > 127.0f) y = 127.0f;
-            if (y < -128.0f) y = -128.0f;
-            q[t * d + i] = (int8_t)y;
-        }
-        token_scale[t] = 1.0f / s;
-    }
+    for (int64_t t = 0; t < B; ++t) token_scale[t] = quantize_row(x + t * d, smooth, d, xf, q + t * d);
     free(xf);
     return ORC_OK;
 }
@@ -280,6 +283,39 @@ int orc_dispatch(const orc_cfg* c, const void* quant_out, const float* token_sca
             if (c->quant_mode == 2) recv_scale[row] = token_scale[t];
         }
     }
+    return ORC_OK;
+}
+
+/*
+ * Dispatch with a per-expert smooth scale (scales of shape [E][d], as in the
+ * Ascend example's quant_mode 2 call): each routed copy (t, g) is quantized on
+ * its own,  x_fp32 = fp32(x[t]) * smooth[g], s = 127 / max|x_fp32|,
+ * q = CastToInt8(x_fp32 * s), and written with recv_scale = 1 / s to its row.
+ * Same readings as orc_quantize (row absmax, round half to even, saturation,
+ * amax == 0 or non-finite s -> zeros and scale 0).  quant_mode 2 only.
+ */
+int orc_dispatch_expert_smooth(const orc_cfg* c, const uint16_t* x, const float* smooth,
+                               const int32_t* topk_idx, const int32_t* dst_pos, int8_t* recv_x,
+                               float* recv_scale, int64_t rows) {
+    if (!cfg_ok(c) || c->quant_mode != 2 || !x || !smooth || !topk_idx || !dst_pos || !recv_x ||
+        !recv_scale)
+        return ORC_BAD_ARG;
+    const int64_t B = c->B, d = c->d, k = c->k, E = c->E;
+    float* xf = (float*)malloc(sizeof(float) * (size_t)d);
+    if (!xf) return ORC_BAD_ARG;
+    for (int64_t t = 0; t < B; ++t) {
+        for (int64_t j = 0; j < k; ++j) {
+            const int64_t row = dst_pos[t * k + j];
+            const int64_t g = topk_idx[t * k + j];
+            if (row < 0) continue;
+            if (g < 0 || g >= E || row >= rows) {
+                free(xf);
+                return ORC_BAD_ARG;
+            }
+            recv_scale[row] = quantize_row(x + t * d, smooth + g * d, d, xf, recv_x + row * d);
+        }
+    }
+    free(xf);
     return ORC_OK;
 }
 

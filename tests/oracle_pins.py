@@ -482,6 +482,39 @@ def pin_quant_inv_order(lib):
     return fails
 
 
+def pin_expert_smooth(lib):
+    """Per-expert smooth scale: against the brute force per routed copy, and the
+    closed form that identical expert rows reproduce the per-token [d] result."""
+    fails = []
+    rng = np.random.default_rng(21)
+    B, d, k, P, M, E = 10, 32, 3, 2, 5, 6
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(B)]).astype(np.int32)
+    idx[3, 1] = -1
+    x = _torch_bf16(rng.standard_normal((B, d)).astype(np.float32))
+    x[4] = 0
+    smooth = rng.uniform(0.25, 4.0, (E, d)).astype(np.float32)
+    cfg = oracle.make_cfg(B, d, k, P, M, E, 0, 0, 0, 2)
+    lay = oracle.layout(cfg, idx, lib=lib)
+    rows = E * P * M
+    rx, rsc = oracle.dispatch_expert_smooth(cfg, x, smooth, idx, lay["dst_pos"], rows, lib=lib)
+    for t in range(B):
+        for j in range(k):
+            row = lay["dst_pos"][t, j]
+            if row < 0:
+                continue
+            bq, binv = brute.quantize_row(x[t].tolist(), smooth[idx[t, j]].tolist())
+            if rx[row].tolist() != bq or struct.pack("<f", rsc[row]) != struct.pack("<f", binv):
+                fails.append("expert smooth: copy (%d, %d) differs from brute force" % (t, j))
+                return fails
+    same = np.tile(smooth[:1], (E, 1))
+    rx2, rsc2 = oracle.dispatch_expert_smooth(cfg, x, same, idx, lay["dst_pos"], rows, lib=lib)
+    q, ts = oracle.quantize(cfg, x, smooth[0], lib=lib)
+    rx3, rsc3 = oracle.dispatch(cfg, q, ts, lay["dst_pos"], rows, lib=lib)
+    if not (np.array_equal(rx2, rx3) and np.array_equal(rsc2.view(np.uint32), rsc3.view(np.uint32))):
+        fails.append("expert smooth with identical rows differs from the per-token scale")
+    return fails
+
+
 # ----------------------------------------------------------------------------- scatter
 
 
@@ -640,6 +673,7 @@ ALL_PINS = [
     pin_quant_properties,
     pin_quant_ties,
     pin_quant_inv_order,
+    pin_expert_smooth,
     pin_dispatch_brute,
     pin_combine_brute,
     pin_combine_closed_forms,

@@ -20,12 +20,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # (name, exact source text, replacement)
 MUTANTS = [
-    ("scale_amax_over_127", "token_scale[t] = 1.0f / s;", "token_scale[t] = amax / 127.0f;"),
+    ("scale_amax_over_127", "return 1.0f / s;", "return amax / 127.0f;"),
     ("round_half_away", "float y = nearbyintf(xf[i] * s);", "float y = roundf(xf[i] * s);"),
     ("round_truncate", "float y = nearbyintf(xf[i] * s);", "float y = truncf(xf[i] * s);"),
     ("signed_max_not_abs", "if (a > amax) amax = a;", "if (v > amax) amax = v;"),
     ("smooth_dropped", "if (smooth) v = v * smooth[i];", "(void)smooth;"),
-    ("zero_row_scale_one", "token_scale[t] = 0.0f;", "token_scale[t] = 1.0f;"),
+    ("zero_row_scale_one", "return 0.0f;\n    }\n    for", "return 1.0f;\n    }\n    for"),
     ("unfused_accumulate", "acc = fmaf(w, e, acc);", "acc = acc + w * e;"),
     ("const_sign", "e = p1 + p2;", "e = p1 - p2;"),
     ("const_operand", "float p2 = bf16_to_f32(a2[ci * d + i]) * bf16_to_f32(v[ci * d + i]);",
@@ -51,6 +51,8 @@ MUTANTS = [
      "for (int64_t j = 0; j < k - 1; ++j) {\n                int64_t g = topk_idx[t * k + j];\n                float w"),
     ("scatter_scale_dropped", "if (c->quant_mode == 2) recv_scale[row] = token_scale[t];",
      "(void)recv_scale;"),
+    ("expert_smooth_wrong_row", "smooth + g * d, d, xf", "smooth + ((g + 1) % E) * d, d, xf"),
+    ("expert_smooth_token_row", "quantize_row(x + t * d, smooth + g", "quantize_row(x + (t ^ 1) % B * d, smooth + g"),
     ("packed_rank_prefix_dropped", "for (int64_t rr = 0; rr < r; ++rr) base += recv_count[g * P + rr];",
      "for (int64_t rr = 0; rr < 0; ++rr) base += recv_count[g * P + rr];"),
     ("packed_rank_prefix_inclusive", "for (int64_t rr = 0; rr < r; ++rr) base += recv_count[g * P + rr];",
