@@ -53,6 +53,10 @@ def load(path=None):
     lib.orc_receive_rows.restype = i64
     lib.orc_dispatch_expert_smooth.argtypes = [P, P, P, P, P, P, P, i64]
     lib.orc_dispatch_expert_smooth.restype = ctypes.c_int
+    lib.orc_layout_active.argtypes = [P] * 9
+    lib.orc_layout_active.restype = ctypes.c_int
+    lib.orc_combine_active.argtypes = [P, P, i64, P, P, P, P, P, P, P, P, P]
+    lib.orc_combine_active.restype = ctypes.c_int
     if path == _build.LIB or os.path.abspath(path) == os.path.abspath(_build.LIB):
         _lib, _lib_path = lib, _build.LIB
     return lib
@@ -84,9 +88,10 @@ def _check(rc, name):
         raise ValueError("oracle %s rejected its arguments (status %d)" % (name, rc))
 
 
-def layout(cfg, topk_idx, lib=None):
+def layout(cfg, topk_idx, lib=None, active=None):
     """Returns dict(expert_count, expert_offset, recv_count [E,P], dst_pos [B,k],
-    recv_src [rows], err); rows = E*P*M (low-latency) or B*k (packed)."""
+    recv_src [rows], err); rows = E*P*M (low-latency) or B*k (packed).
+    active: optional [B] x_active_mask (nonzero = active)."""
     lib = lib or load()
     E_tot = cfg.E + cfg.n_zero + cfg.n_copy + cfg.n_const
     idx = _c(topk_idx, np.int32)
@@ -98,20 +103,25 @@ def layout(cfg, topk_idx, lib=None):
         recv_src=np.zeros(receive_rows(cfg, lib), np.int32),
     )
     err = np.zeros(1, np.uint32)
-    rc = lib.orc_layout(ctypes.byref(cfg), _ptr(idx), _ptr(out["expert_count"]),
-                        _ptr(out["expert_offset"]), _ptr(out["recv_count"]),
-                        _ptr(out["dst_pos"]), _ptr(out["recv_src"]), _ptr(err))
+    act = None if active is None else (np.asarray(active) != 0).astype(np.uint8)
+    rc = lib.orc_layout_active(ctypes.byref(cfg), _ptr(idx), _ptr(act), _ptr(out["expert_count"]),
+                               _ptr(out["expert_offset"]), _ptr(out["recv_count"]),
+                               _ptr(out["dst_pos"]), _ptr(out["recv_src"]), _ptr(err))
     _check(rc, "layout")
     out["err"] = int(err[0])
     return out
 
 
 def quantize(cfg, x_bits, smooth=None, lib=None):
-    """Returns (quant_out [B,d] int8 or uint16, token_scale [B] float32 or None)."""
+    """Returns (quant_out [B,d] int8 or uint16, token_scale [B] float32 or None);
+    quant_mode 1 (static cast) returns no scale."""
     lib = lib or load()
     x = _c(x_bits, np.uint16)
     ss = _c(smooth, np.float32)
-    if cfg.quant_mode == 2:
+    if cfg.quant_mode == 1:
+        q = np.zeros((cfg.B, cfg.d), np.int8)
+        sc = None
+    elif cfg.quant_mode == 2:
         q = np.zeros((cfg.B, cfg.d), np.int8)
         sc = np.zeros(cfg.B, np.float32)
     else:
@@ -139,11 +149,11 @@ def dispatch(cfg, quant_out, token_scale, dst_pos, rows, lib=None):
 
 def dispatch_expert_smooth(cfg, x_bits, smooth_E, topk_idx, dst_pos, rows, lib=None):
     """Per-copy quantization with a [E, d] smooth scale, scattered to `rows` receive
-    rows.  Returns (recv_x int8 [rows, d], recv_scale float32 [rows]); rows no pick
-    maps to stay zero."""
+    rows.  Returns (recv_x int8 [rows, d], recv_scale float32 [rows], or None in
+    quant_mode 1); rows no pick maps to stay zero."""
     lib = lib or load()
     recv_x = np.zeros((rows, cfg.d), np.int8)
-    recv_scale = np.zeros(rows, np.float32)
+    recv_scale = np.zeros(rows, np.float32) if cfg.quant_mode == 2 else None
     rc = lib.orc_dispatch_expert_smooth(ctypes.byref(cfg), _ptr(_c(x_bits, np.uint16)),
                                         _ptr(_c(smooth_E, np.float32)), _ptr(_c(topk_idx, np.int32)),
                                         _ptr(_c(dst_pos, np.int32)), _ptr(recv_x), _ptr(recv_scale),
@@ -153,16 +163,18 @@ def dispatch_expert_smooth(cfg, x_bits, smooth_E, topk_idx, dst_pos, rows, lib=N
 
 
 def combine(cfg, expert_out, topk_idx, topk_weights, dst_pos, ori_x=None, a1=None, a2=None,
-            v=None, lib=None):
-    """Returns y [B,d] as bf16 bits (uint16).  expert_out is [rows, d] bf16 bits."""
+            v=None, lib=None, active=None):
+    """Returns y [B,d] as bf16 bits (uint16).  expert_out is [rows, d] bf16 bits;
+    active: optional [B] x_active_mask (inactive tokens give +0)."""
     lib = lib or load()
     eo = _c(expert_out, np.uint16)
     rows = 0 if eo is None else eo.shape[0]
     y = np.zeros((cfg.B, cfg.d), np.uint16)
-    rc = lib.orc_combine(ctypes.byref(cfg), _ptr(eo), rows, _ptr(_c(topk_idx, np.int32)),
-                         _ptr(_c(topk_weights, np.float32)), _ptr(_c(dst_pos, np.int32)),
-                         _ptr(_c(ori_x, np.uint16)), _ptr(_c(a1, np.uint16)),
-                         _ptr(_c(a2, np.uint16)), _ptr(_c(v, np.uint16)), _ptr(y))
+    act = None if active is None else (np.asarray(active) != 0).astype(np.uint8)
+    rc = lib.orc_combine_active(ctypes.byref(cfg), _ptr(eo), rows, _ptr(_c(topk_idx, np.int32)),
+                                _ptr(_c(topk_weights, np.float32)), _ptr(_c(dst_pos, np.int32)),
+                                _ptr(_c(ori_x, np.uint16)), _ptr(_c(a1, np.uint16)),
+                                _ptr(_c(a2, np.uint16)), _ptr(_c(v, np.uint16)), _ptr(act), _ptr(y))
     _check(rc, "combine")
     return y
 

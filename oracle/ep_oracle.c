@@ -18,6 +18,9 @@
  *    "Deterministic Computation: defaults to a deterministic computation".
  *  - same page, Example: special-expert ids follow the routed ones
  *    (num_experts = 32 with one zero and one copy expert uses ids 32 and 33).
+ *  - same page, Formula, non-dynamic case: quant_mode 1 (any mode other than 0
+ *    and 2) is the static cast CastToInt8(CastToFp32(x) * scales), no scale sent.
+ *  - same page, Prototype: the optional per-token x_active_mask.
  *  - DeepEP issue #84 "Profiling dispatch_t for low-latency kernel dispatch
  *    bandwidth", masking experiment: expert g lives on rank g / (E / P) and a
  *    pick set to -1 sends nothing.
@@ -35,7 +38,11 @@
  *    the constant expert is alpha1 * x + alpha2 * v in fp32 (two rounded products,
  *    one rounded sum), no bf16 rounding before weighting;
  *  - combine accumulates acc = fma(w_j, e_j, acc) in fp32 in pick order j and
- *    rounds once to bf16 (nearest even).
+ *    rounds once to bf16 (nearest even);
+ *  - static quantization (mode 1) with no scale given multiplies by nothing;
+ *  - x_active_mask: a token whose entry is 0 takes no part at all, as if every
+ *    pick of it were -1: no receive row, not counted (special experts included),
+ *    no error bits for its ids, and combine returns +0 for it.
  *
  * Build: gcc -std=c11 -O2 -ffp-contract=off -fPIC -shared (no fast-math).
  */
@@ -63,7 +70,7 @@ typedef struct {
     int32_t n_zero;     /* zero experts */
     int32_t n_copy;     /* copy experts */
     int32_t n_const;    /* constant experts */
-    int32_t quant_mode; /* 0: bf16 pass-through, 2: dynamic int8 */
+    int32_t quant_mode; /* 0: bf16 pass-through, 1: static int8, 2: dynamic int8 */
     int32_t layout;     /* 0: low-latency rows, 1: packed rows */
 } orc_cfg;
 
@@ -97,7 +104,7 @@ static int cfg_ok(const orc_cfg* c) {
     if (c->B % c->P != 0 || c->E % c->P != 0) return 0;
     if (c->layout != 0 && c->layout != 1) return 0;
     if (c->layout == 0 && c->B / c->P > c->M) return 0;
-    if (c->quant_mode != 0 && c->quant_mode != 2) return 0;
+    if (c->quant_mode < 0 || c->quant_mode > 2) return 0;
     return 1;
 }
 
@@ -130,10 +137,11 @@ void orc_f32_to_bf16_n(const float* in, uint16_t* out, int64_t n) {
  * dst_pos       [B][k]               global receive row, or -1 if not routed
  * recv_src      [rows]               source token of each received row; -1 in
  *                                    rows nobody wrote (rows = E*P*M or B*k)
+ * active        [B] or NULL          x_active_mask: tokens with 0 are skipped
  */
-int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
-               int32_t* expert_offset, int32_t* recv_count, int32_t* dst_pos,
-               int32_t* recv_src, uint32_t* err_bits) {
+int orc_layout_active(const orc_cfg* c, const int32_t* topk_idx, const uint8_t* active,
+                      int32_t* expert_count, int32_t* expert_offset, int32_t* recv_count,
+                      int32_t* dst_pos, int32_t* recv_src, uint32_t* err_bits) {
     if (!cfg_ok(c) || !topk_idx || !expert_count || !expert_offset || !recv_count ||
         !dst_pos || !recv_src || !err_bits)
         return ORC_BAD_ARG;
@@ -149,6 +157,10 @@ int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
 
     for (int64_t r = 0; r < P; ++r) {
         for (int64_t t = r * T; t < (r + 1) * T; ++t) {
+            if (active && !active[t]) {              /* inactive token: nothing at all */
+                for (int64_t j = 0; j < k; ++j) dst_pos[t * k + j] = -1;
+                continue;
+            }
             for (int64_t j = 0; j < k; ++j) {
                 int64_t g = topk_idx[t * k + j];
                 dst_pos[t * k + j] = -1;
@@ -211,9 +223,30 @@ int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
     return ORC_OK;
 }
 
+int orc_layout(const orc_cfg* c, const int32_t* topk_idx, int32_t* expert_count,
+               int32_t* expert_offset, int32_t* recv_count, int32_t* dst_pos,
+               int32_t* recv_src, uint32_t* err_bits) {
+    return orc_layout_active(c, topk_idx, NULL, expert_count, expert_offset, recv_count, dst_pos,
+                             recv_src, err_bits);
+}
+
+/* Static cast of one row (quant_mode 1): q = CastToInt8(fp32(x) (* scales)), round
+ * half to even, saturate; no scale is derived. */
+static void cast_row_static(const uint16_t* x, const float* scales, int64_t d, int8_t* q) {
+    for (int64_t i = 0; i < d; ++i) {
+        float v = bf16_to_f32(x[i]);
+        if (scales) v = v * scales[i];
+        float y = nearbyintf(v);
+        if (y > 127.0f) y = 127.0f;
+        else if (y < -128.0f) y = -128.0f;
+        q[i] = (int8_t)y;
+    }
+}
+
 /*
  * Per-token quantization.
  *  quant_mode 0: quant_out = x (bf16 bits copied), token_scale untouched.
+ *  quant_mode 1: q = CastToInt8(fp32(x) * smooth), token_scale untouched.
  *  quant_mode 2: x_fp32 = fp32(x) * smooth, s = 127 / max|x_fp32|,
  *                q = CastToInt8(x_fp32 * s), token_scale = 1 / s.
  * smooth is a [d] fp32 vector or NULL (NULL means no multiply at all).
@@ -252,8 +285,12 @@ int orc_quantize(const orc_cfg* c, const uint16_t* x, const float* smooth, void*
         for (int64_t i = 0; i < B * d; ++i) out[i] = x[i];
         return ORC_OK;
     }
-    if (!token_scale) return ORC_BAD_ARG;
     int8_t* q = (int8_t*)quant_out;
+    if (c->quant_mode == 1) {
+        for (int64_t t = 0; t < B; ++t) cast_row_static(x + t * d, smooth, d, q + t * d);
+        return ORC_OK;
+    }
+    if (!token_scale) return ORC_BAD_ARG;
     float* xf = (float*)malloc(sizeof(float) * (size_t)d);
     if (!xf) return ORC_BAD_ARG;
     for (int64_t t = 0; t < B; ++t) token_scale[t] = quantize_row(x + t * d, smooth, d, xf, q + t * d);
@@ -272,7 +309,7 @@ int orc_dispatch(const orc_cfg* c, const void* quant_out, const float* token_sca
     if (!cfg_ok(c) || !quant_out || !dst_pos || !recv_x) return ORC_BAD_ARG;
     if (c->quant_mode == 2 && (!token_scale || !recv_scale)) return ORC_BAD_ARG;
     const int64_t B = c->B, d = c->d, k = c->k;
-    const int64_t esz = (c->quant_mode == 2) ? 1 : 2;
+    const int64_t esz = (c->quant_mode != 0) ? 1 : 2;
     for (int64_t t = 0; t < B; ++t) {
         for (int64_t j = 0; j < k; ++j) {
             int64_t row = dst_pos[t * k + j];
@@ -292,14 +329,16 @@ int orc_dispatch(const orc_cfg* c, const void* quant_out, const float* token_sca
  * its own,  x_fp32 = fp32(x[t]) * smooth[g], s = 127 / max|x_fp32|,
  * q = CastToInt8(x_fp32 * s), and written with recv_scale = 1 / s to its row.
  * Same readings as orc_quantize (row absmax, round half to even, saturation,
- * amax == 0 or non-finite s -> zeros and scale 0).  quant_mode 2 only.
+ * amax == 0 or non-finite s -> zeros and scale 0).  In quant_mode 1 each copy is
+ * the static cast with its expert's row, q = CastToInt8(fp32(x[t]) * smooth[g]),
+ * and recv_scale is not used.
  */
 int orc_dispatch_expert_smooth(const orc_cfg* c, const uint16_t* x, const float* smooth,
                                const int32_t* topk_idx, const int32_t* dst_pos, int8_t* recv_x,
                                float* recv_scale, int64_t rows) {
-    if (!cfg_ok(c) || c->quant_mode != 2 || !x || !smooth || !topk_idx || !dst_pos || !recv_x ||
-        !recv_scale)
+    if (!cfg_ok(c) || c->quant_mode == 0 || !x || !smooth || !topk_idx || !dst_pos || !recv_x)
         return ORC_BAD_ARG;
+    if (c->quant_mode == 2 && !recv_scale) return ORC_BAD_ARG;
     const int64_t B = c->B, d = c->d, k = c->k, E = c->E;
     float* xf = (float*)malloc(sizeof(float) * (size_t)d);
     if (!xf) return ORC_BAD_ARG;
@@ -312,7 +351,10 @@ int orc_dispatch_expert_smooth(const orc_cfg* c, const uint16_t* x, const float*
                 free(xf);
                 return ORC_BAD_ARG;
             }
-            recv_scale[row] = quantize_row(x + t * d, smooth + g * d, d, xf, recv_x + row * d);
+            if (c->quant_mode == 1)
+                cast_row_static(x + t * d, smooth + g * d, d, recv_x + row * d);
+            else
+                recv_scale[row] = quantize_row(x + t * d, smooth + g * d, d, xf, recv_x + row * d);
         }
     }
     free(xf);
@@ -326,21 +368,23 @@ int orc_dispatch_expert_smooth(const orc_cfg* c, const uint16_t* x, const float*
  *   -1, zero expert, bad id, or routed id with dst_pos < 0 : the term is skipped
  *   copy expert c              : e = fp32(ori_x[t])
  *   const expert c             : e = fp32(a1[c]) * fp32(ori_x[t]) + fp32(a2[c]) * fp32(v[c])
- * expert_out has `rows` rows of d bf16 values.
+ * expert_out has `rows` rows of d bf16 values.  active ([B] or NULL): a token
+ * whose entry is 0 has every term skipped, so y[t] = +0.
  */
-int orc_combine(const orc_cfg* c, const uint16_t* expert_out, int64_t rows,
-                const int32_t* topk_idx, const float* topk_weights, const int32_t* dst_pos,
-                const uint16_t* ori_x, const uint16_t* a1, const uint16_t* a2,
-                const uint16_t* v, uint16_t* y) {
+int orc_combine_active(const orc_cfg* c, const uint16_t* expert_out, int64_t rows,
+                       const int32_t* topk_idx, const float* topk_weights, const int32_t* dst_pos,
+                       const uint16_t* ori_x, const uint16_t* a1, const uint16_t* a2,
+                       const uint16_t* v, const uint8_t* active, uint16_t* y) {
     if (!cfg_ok(c) || !topk_idx || !topk_weights || !dst_pos || !y) return ORC_BAD_ARG;
     const int64_t B = c->B, d = c->d, k = c->k, E = c->E;
     const int64_t Z = c->n_zero, C = c->n_copy, K = c->n_const;
     if ((C + K) > 0 && !ori_x) return ORC_BAD_ARG;
     if (K > 0 && (!a1 || !a2 || !v)) return ORC_BAD_ARG;
     for (int64_t t = 0; t < B; ++t) {
+        const int64_t k_t = (active && !active[t]) ? 0 : k;
         for (int64_t i = 0; i < d; ++i) {
             float acc = 0.0f;
-            for (int64_t j = 0; j < k; ++j) {
+            for (int64_t j = 0; j < k_t; ++j) {
                 int64_t g = topk_idx[t * k + j];
                 float w = topk_weights[t * k + j];
                 float e;
@@ -365,4 +409,12 @@ int orc_combine(const orc_cfg* c, const uint16_t* expert_out, int64_t rows,
         }
     }
     return ORC_OK;
+}
+
+int orc_combine(const orc_cfg* c, const uint16_t* expert_out, int64_t rows,
+                const int32_t* topk_idx, const float* topk_weights, const int32_t* dst_pos,
+                const uint16_t* ori_x, const uint16_t* a1, const uint16_t* a2,
+                const uint16_t* v, uint16_t* y) {
+    return orc_combine_active(c, expert_out, rows, topk_idx, topk_weights, dst_pos, ori_x, a1, a2,
+                              v, NULL, y);
 }

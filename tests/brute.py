@@ -78,11 +78,12 @@ def float_to_bf16_bits(f):
     return bits >> 16
 
 
-def layout(topk_idx, B, k, P, M, E, n_special, packed=False):
+def layout(topk_idx, B, k, P, M, E, n_special, packed=False, active=None):
     """Returns (expert_count, recv_count[g][r], dst_pos[t][j], recv_src dict row->t, err).
     packed: rows of expert g come after every pick of a lower expert id, and within
     g the rows of rank r after those of lower ranks (contiguous per expert, then
-    per rank); otherwise row = g*P*M + r*M + slot."""
+    per rank); otherwise row = g*P*M + r*M + slot.  active: optional per-token
+    flags; a token whose flag is false is not looked at."""
     E_tot = E + n_special
     T = B // P
     expert_count = [0] * E_tot
@@ -90,9 +91,14 @@ def layout(topk_idx, B, k, P, M, E, n_special, packed=False):
     dst_pos = [[-1] * k for _ in range(B)]
     recv_src = {}
     err = 0
+    def on(t):
+        return active is None or bool(active[t])
+
     for t in range(B):
         r = t // T
         seen = set()
+        if not on(t):
+            continue
         for j in range(k):
             g = int(topk_idx[t][j])
             if g == -1:
@@ -111,7 +117,7 @@ def layout(topk_idx, B, k, P, M, E, n_special, packed=False):
             slot = 0
             for t2 in range(r * T, t):
                 row_ids = [int(v) for v in topk_idx[t2]]
-                if g in row_ids:
+                if on(t2) and g in row_ids:
                     slot += 1
             if packed:
                 dst_pos[t][j] = (g, r, slot)  # resolved below, once all counts are known
@@ -157,6 +163,17 @@ def quantize_row(xbits, smooth=None):
         z = round(f32(v * s))  # Python round(): half to even
         q.append(max(-128, min(127, z)))
     return q, f32(1.0 / s)
+
+
+def cast_static_row(xbits, scales=None):
+    """Static int8 cast of one row (quant_mode 1): q = clamp(round_half_even(x * scale))."""
+    q = []
+    for i, h in enumerate(xbits):
+        v = bf16_bits_to_float(h)
+        if scales is not None:
+            v = f32(v * float(scales[i]))
+        q.append(max(-128, min(127, round(v))))
+    return q
 
 
 def combine_token(d, picks, weights, E, Z, C, K, expert_row, ori_row, a1, a2, v):

@@ -661,6 +661,140 @@ def pin_combine_closed_forms(lib):
     return fails
 
 
+# ----------------------------------------------------------------------------- x_active_mask
+
+
+def pin_active_mask(lib):
+    """x_active_mask: brute force (inactive tokens not looked at, in low-latency and
+    packed rows), the all-ones mask equals no mask, the all-zeros mask routes and
+    counts nothing and flags no bad id, and combine gives +0 for inactive tokens
+    and, for active ones, what it gives without the mask."""
+    fails = []
+    rng = np.random.default_rng(31)
+    for trial in range(8):
+        P = int(rng.integers(1, 4))
+        T = int(rng.integers(2, 7))
+        B, M = P * T, T + int(rng.integers(0, 2))
+        L = int(rng.integers(1, 4))
+        E = L * P
+        Z, C, K = (int(v) for v in rng.integers(0, 2, 3))
+        E_tot = E + Z + C + K
+        k = int(rng.integers(1, min(5, E_tot) + 1))
+        idx = np.stack([rng.permutation(E_tot)[:k] for _ in range(B)]).astype(np.int32)
+        if trial % 2:
+            idx[rng.integers(0, B), 0] = E_tot + 1       # a bad id (flagged only if active)
+        act = (rng.random(B) < 0.6).astype(np.uint8)
+        packed = trial % 4 >= 2
+        cfg = oracle.make_cfg(B, 16, k, P, M, E, Z, C, K, 0, layout=int(packed))
+        out = oracle.layout(cfg, idx, lib=lib, active=act)
+        ref = brute.layout(idx.tolist(), B, k, P, M, E, Z + C + K, packed=packed, active=act.tolist())
+        rows = oracle.receive_rows(cfg, lib)
+        fails += _compare_layout("active mask trial %d" % trial, out, ref, B, k, P, M, E, rows=rows)
+        full = oracle.layout(cfg, idx, lib=lib, active=np.ones(B, np.uint8))
+        plain = oracle.layout(cfg, idx, lib=lib)
+        if any(not np.array_equal(full[n], plain[n]) for n in ("expert_count", "dst_pos", "recv_src")) \
+                or full["err"] != plain["err"]:
+            fails.append("active mask of ones differs from no mask (trial %d)" % trial)
+        none = oracle.layout(cfg, idx, lib=lib, active=np.zeros(B, np.uint8))
+        if none["expert_count"].any() or (none["dst_pos"] != -1).any() or none["err"]:
+            fails.append("active mask of zeros still routes, counts or flags (trial %d)" % trial)
+        if fails:
+            return fails
+    # combine
+    B, d, k, P, M, E, Z, C, K = 12, 16, 3, 2, 6, 6, 1, 1, 1
+    E_tot = E + Z + C + K
+    idx = np.stack([rng.permutation(E_tot)[:k] for _ in range(B)]).astype(np.int32)
+    act = np.array([1, 0, 1, 1, 0, 1, 0, 1, 1, 0, 1, 1], np.uint8)
+    cfg = oracle.make_cfg(B, d, k, P, M, E, Z, C, K, 0)
+    lay = oracle.layout(cfg, idx, lib=lib, active=act)
+    eo = _torch_bf16(rng.standard_normal((E * P * M, d)).astype(np.float32))
+    x = _torch_bf16(rng.standard_normal((B, d)).astype(np.float32))
+    a1 = _torch_bf16(rng.random((K, d)).astype(np.float32))
+    a2 = _torch_bf16(rng.random((K, d)).astype(np.float32))
+    v = _torch_bf16(rng.standard_normal((K, d)).astype(np.float32))
+    wts = rng.standard_normal((B, k)).astype(np.float32)
+    y = oracle.combine(cfg, eo, idx, wts, lay["dst_pos"], x, a1, a2, v, lib=lib, active=act)
+    y0 = oracle.combine(cfg, eo, idx, wts, lay["dst_pos"], x, a1, a2, v, lib=lib)
+    if np.any(y[act == 0] != 0):
+        fails.append("combine: inactive tokens are not +0")
+    if not np.array_equal(y[act == 1], y0[act == 1]):
+        fails.append("combine: active tokens differ from the unmasked combine")
+    for t in np.nonzero(act)[0][:3]:
+        picks = [(int(idx[t, j]), int(lay["dst_pos"][t, j])) for j in range(k)]
+        want = brute.combine_token(d, picks, wts[t].tolist(), E, Z, C, K, lambda r: eo[r].tolist(),
+                                   x[t].tolist(), a1.tolist(), a2.tolist(), v.tolist())
+        if y[t].tolist() != want:
+            fails.append("combine: active token %d differs from brute force" % t)
+    return fails
+
+
+# ----------------------------------------------------------------------------- static quantization
+
+
+def pin_static_quant(lib):
+    """quant_mode 1, CastToInt8(CastToFp32(x) * scales): brute force with and
+    without scales, exact closed forms (integers, ties, saturation), the per-copy
+    form with an [E, d] scale, and the scatter carrying no scale."""
+    fails = []
+    rng = np.random.default_rng(41)
+    B, d = 6, 40
+    x = _torch_bf16((rng.standard_normal((B, d)) * 40).astype(np.float32))
+    for smooth in (None, rng.uniform(0.25, 4.0, d).astype(np.float32)):
+        cfg = oracle.make_cfg(B, d, 1, 1, B, 1, 0, 0, 0, 1)
+        q, sc = oracle.quantize(cfg, x, smooth, lib=lib)
+        if sc is not None:
+            fails.append("static cast returned a scale")
+        for t in range(B):
+            want = brute.cast_static_row(x[t].tolist(), None if smooth is None else smooth.tolist())
+            if q[t].tolist() != want:
+                fails.append("static cast row %d (scales %s) differs from brute force"
+                             % (t, "none" if smooth is None else "set"))
+                return fails
+    # integers pass through, x.5 ties go to even, beyond the int8 range saturates
+    vals = np.array([0, 1, -1, 2.5, 3.5, -2.5, -0.5, 0.5, 126, 127, 127.5, 128, 300,
+                     -128, -128.5, -129, -300, 1.5, -1.5, 64.25], np.float32)
+    want = [0, 1, -1, 2, 4, -2, 0, 0, 126, 127, 127, 127, 127, -128, -128, -128, -128, 2, -2, 64]
+    cfg = oracle.make_cfg(1, 32, 1, 1, 1, 1, 0, 0, 0, 1)
+    xv = np.zeros((1, 32), np.float32)
+    xv[0, :vals.size] = vals
+    q, _ = oracle.quantize(cfg, _torch_bf16(xv), None, lib=lib)
+    if q[0, :vals.size].tolist() != want:
+        fails.append("static cast closed forms: got %s, want %s" % (q[0, :vals.size].tolist(), want))
+    # a power-of-two scale is exact: q(x, 2^-3) = q(x / 8)
+    q8, _ = oracle.quantize(cfg, _torch_bf16(xv), np.full(32, 0.125, np.float32), lib=lib)
+    qd, _ = oracle.quantize(cfg, _torch_bf16(xv / 8), None, lib=lib)
+    if not np.array_equal(q8, qd):
+        fails.append("static cast with scale 2^-3 differs from the cast of x / 8")
+    # per-copy with an [E, d] scale, scattered; the scatter carries no scale
+    Bp, k, P, E = 8, 3, 2, 6
+    M = Bp // P
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(Bp)]).astype(np.int32)
+    xs = _torch_bf16((rng.standard_normal((Bp, d)) * 30).astype(np.float32))
+    sm = rng.uniform(0.25, 4.0, (E, d)).astype(np.float32)
+    cfg = oracle.make_cfg(Bp, d, k, P, M, E, 0, 0, 0, 1)
+    lay = oracle.layout(cfg, idx, lib=lib)
+    rows = E * P * M
+    rx, rsc = oracle.dispatch_expert_smooth(cfg, xs, sm, idx, lay["dst_pos"], rows, lib=lib)
+    if rsc is not None:
+        fails.append("static per-copy dispatch returned scales")
+    for t in range(Bp):
+        for j in range(k):
+            row = lay["dst_pos"][t, j]
+            if rx[row].tolist() != brute.cast_static_row(xs[t].tolist(), sm[idx[t, j]].tolist()):
+                fails.append("static per-copy row (%d, %d) differs from brute force" % (t, j))
+                return fails
+    q, _ = oracle.quantize(cfg, xs, sm[2], lib=lib)
+    rx2, rs2 = oracle.dispatch(cfg, q, None, lay["dst_pos"], rows, lib=lib)
+    if rs2 is not None or rx2.dtype != np.int8:
+        fails.append("static scatter: wrong payload type or a scale")
+    for t in range(Bp):
+        for j in range(k):
+            if rx2[lay["dst_pos"][t, j]].tolist() != q[t].tolist():
+                fails.append("static scatter: row (%d, %d) is not the token's cast" % (t, j))
+                return fails
+    return fails
+
+
 ALL_PINS = [
     pin_bf16_format,
     pin_layout_golden,
@@ -677,4 +811,6 @@ ALL_PINS = [
     pin_dispatch_brute,
     pin_combine_brute,
     pin_combine_closed_forms,
+    pin_active_mask,
+    pin_static_quant,
 ]

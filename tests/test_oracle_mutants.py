@@ -47,12 +47,20 @@ MUTANTS = [
      "continue;"),
     ("bf16_ties_away", "u = u + 0x7fffu + keep_lsb;", "u = u + 0x8000u + 0 * keep_lsb;"),
     ("bf16_truncate", "u = u + 0x7fffu + keep_lsb;", "u = u + 0 * keep_lsb;"),
-    ("last_pick_dropped", "for (int64_t j = 0; j < k; ++j) {\n                int64_t g = topk_idx[t * k + j];\n                float w",
-     "for (int64_t j = 0; j < k - 1; ++j) {\n                int64_t g = topk_idx[t * k + j];\n                float w"),
+    ("last_pick_dropped", "for (int64_t j = 0; j < k_t; ++j) {", "for (int64_t j = 0; j < k_t - 1; ++j) {"),
     ("scatter_scale_dropped", "if (c->quant_mode == 2) recv_scale[row] = token_scale[t];",
      "(void)recv_scale;"),
     ("expert_smooth_wrong_row", "smooth + g * d, d, xf", "smooth + ((g + 1) % E) * d, d, xf"),
     ("expert_smooth_token_row", "quantize_row(x + t * d, smooth + g", "quantize_row(x + (t ^ 1) % B * d, smooth + g"),
+    ("active_ignored_in_layout", "if (active && !active[t]) {", "if (0 && active && !active[t]) {"),
+    ("active_inverted_in_layout", "if (active && !active[t]) {", "if (active && active[t]) {"),
+    ("active_slot_counts_inactive", "for (int64_t j = 0; j < k; ++j) dst_pos[t * k + j] = -1;\n                continue;",
+     "for (int64_t j = 0; j < k; ++j) dst_pos[t * k + j] = -1;"),
+    ("active_ignored_in_combine", "(active && !active[t]) ? 0 : k;", "k;"),
+    ("static_round_away", "float y = nearbyintf(v);", "float y = roundf(v);"),
+    ("static_scale_dropped", "if (scales) v = v * scales[i];", "(void)scales;"),
+    ("static_wraps", "if (y > 127.0f) y = 127.0f;\n        else", "if (y > 127.0f) y = y - 256.0f;\n        else"),
+    ("static_copy_first_row", "cast_row_static(x + t * d, smooth + g * d", "cast_row_static(x + t * d, smooth + 0 * g * d"),
     ("packed_rank_prefix_dropped", "for (int64_t rr = 0; rr < r; ++rr) base += recv_count[g * P + rr];",
      "for (int64_t rr = 0; rr < 0; ++rr) base += recv_count[g * P + rr];"),
     ("packed_rank_prefix_inclusive", "for (int64_t rr = 0; rr < r; ++rr) base += recv_count[g * P + rr];",
