@@ -231,32 +231,39 @@ def oracle_step_sample(w, inp, n_tokens):
     idx = np.ascontiguousarray(inp["topk_idx"][:B])
     x = np.ascontiguousarray(inp["x"][:B])
     wts = np.ascontiguousarray(inp["topk_weights"][:B])
+    act = None if inp.get("active") is None else np.ascontiguousarray(inp["active"][:B])
     t0 = time.perf_counter()
-    lay = oracle.layout(cfg, idx)
-    q, ts = oracle.quantize(cfg, x, inp["smooth"])
+    lay = oracle.layout(cfg, idx, active=act)
     # scatter into a compact receive buffer (one row per routed pick, same bytes)
     dp = lay["dst_pos"]
     compact = np.full(dp.shape, -1, np.int32)
     routed = dp >= 0
     n_r = int(routed.sum())
     compact[routed] = np.arange(n_r, dtype=np.int32)
-    rx, rsc = oracle.dispatch(cfg, q, ts, compact, max(n_r, 1))
+    if w.smooth == "expert":
+        rx, rsc = oracle.dispatch_expert_smooth(cfg, x, inp["smooth"], idx, compact, max(n_r, 1))
+    else:
+        q, ts = oracle.quantize(cfg, x, inp["smooth"])
+        rx, rsc = oracle.dispatch(cfg, q, ts, compact, max(n_r, 1))
     t1 = time.perf_counter()
     # stand-in expert outputs (bf16 bit patterns) for combine; not part of the
     # method and not timed
-    if w.quant_mode == 2:
+    if w.quant_mode != 0:
         eo = np.zeros((max(n_r, 1), w.d), np.uint16)
         if n_r:
-            f = rx[:n_r].astype(np.float32) * rsc[:n_r, None]
+            f = rx[:n_r].astype(np.float32)
+            if w.quant_mode == 2:
+                f = f * rsc[:n_r, None]
             eo[:n_r] = (f.view(np.uint32) >> 16).astype(np.uint16)
     else:
         eo = rx
     t2 = time.perf_counter()
-    y = oracle.combine(cfg, eo, idx, wts, compact, x, inp["a1"], inp["a2"], inp["v"])
+    y = oracle.combine(cfg, eo, idx, wts, compact, x, inp["a1"], inp["a2"], inp["v"], active=act)
     t3 = time.perf_counter()
     del y
-    nr, bsp = metrics.routing_counts(w.with_(B=B), idx, n_r)
-    by = metrics.kernel_bytes(w.with_(B=B, P=P, M=M), nr, bsp, smooth=inp["smooth"] is not None)
+    nr, bsp = metrics.routing_counts(w.with_(B=B), idx, n_r, active=act)
+    by = metrics.kernel_bytes(w.with_(B=B, P=P, M=M), nr, bsp, smooth=inp["smooth"] is not None,
+                              masked=act is not None)
     return (t1 - t0) + (t3 - t2), sum(by.values())
 
 
@@ -312,7 +319,7 @@ def run_reference(args):
 def config_dict(w, args):
     return {"workload": w.name, "B": w.B, "d": w.d, "E": w.E, "k": w.k, "P": w.P, "M": w.M,
             "n_zero": w.n_zero, "n_copy": w.n_copy, "n_const": w.n_const,
-            "quant_mode": w.quant_mode, "payload": "int8" if w.quant_mode == 2 else "bf16",
+            "quant_mode": w.quant_mode, "payload": "int8" if w.quant_mode != 0 else "bf16",
             "routing": w.routing, "layout": "low-latency [E, P*M, d]",
             "l2": ("flushed between steps (%d MB memset, outside the step events)" % args.flush_mb)
             if args.flush_mb else "not flushed",
@@ -330,8 +337,8 @@ class Workbench:
         import torch
         from combine_ep_layout_12_b200 import metrics, runner
         self.w, self.device, self.stream = w, device, stream
-        set_bytes = w.rows * w.d * (1 if w.quant_mode == 2 else 2) + w.rows * 12 + 4 * w.B * w.d
-        if w.quant_mode == 2:
+        set_bytes = w.rows * w.d * (1 if w.quant_mode != 0 else 2) + w.rows * 12 + 4 * w.B * w.d
+        if w.quant_mode != 0:
             set_bytes += w.rows * w.d * 2
         free = torch.cuda.mem_get_info(device)[0]
         if set_bytes > 0.9 * free:
@@ -351,20 +358,23 @@ class Workbench:
             assert pipe.buf.check(stream) == 0, "device error bits set"
             dp = pipe.buf.dst_pos
             rows = dp[dp >= 0].long()
-            if w.quant_mode == 2:  # identity expert: expert_out rows = dequantized receive rows
-                deq = pipe.buf.recv_x[rows].float() * pipe.buf.recv_scale[rows].unsqueeze(1)
+            if w.quant_mode != 0:  # identity expert: expert_out rows = dequantized receive rows
+                deq = pipe.buf.recv_x[rows].float()
+                if w.quant_mode == 2:
+                    deq = deq * pipe.buf.recv_scale[rows].unsqueeze(1)
                 pipe.expert_out[rows] = deq.to(torch.bfloat16)
             self.sets.append((pipe, dev_inp))
         torch.cuda.synchronize(device)
         self.n_routed = int((self.sets[0][0].buf.dst_pos >= 0).sum().item())
-        _, b_sp = metrics.routing_counts(w, inp["topk_idx"], self.n_routed)
-        self.kbytes = metrics.kernel_bytes(w, self.n_routed, b_sp, smooth=inp["smooth"] is not None)
+        _, b_sp = metrics.routing_counts(w, inp["topk_idx"], self.n_routed, active=inp.get("active"))
+        self.kbytes = metrics.kernel_bytes(w, self.n_routed, b_sp, smooth=inp["smooth"] is not None,
+                                           masked=inp.get("active") is not None)
         self.step_bytes = sum(self.kbytes.values())
         self.flush = None
         if self.R == 1 and flush_mb:
             self.flush = torch.empty(flush_mb << 20, dtype=torch.uint8, device=device)
         self.S = 2 * self.R if self.R > 1 else 1
-        units = w.d // 16 if w.quant_mode == 2 else w.d // 8
+        units = w.d // 16 if w.quant_mode != 0 else w.d // 8
         # ep_layout_dispatch runs as one grid when T <= 128, k <= 8 and a row fits 128 threads
         self.one_grid = w.B > 0 and w.T <= 128 and w.k <= 8 and units <= 1024
         self.launches_per_step = 2 if self.one_grid else 3
@@ -598,7 +608,7 @@ def run_ours(args):
         "kernels": kernels,
         "layout_then_dispatch_us": 1e3 * kern_ms["layout+dispatch"],
         "layout_dispatch_one_call_us": 1e3 * kern_ms["layout_dispatch"],
-        "comm_gbs_dispatch": wb.n_routed * w.d * (1 if w.quant_mode == 2 else 2)
+        "comm_gbs_dispatch": wb.n_routed * w.d * (1 if w.quant_mode != 0 else 2)
         / (kern_ms["dispatch"] * 1e-3) / 1e9,
         "roofline": roofline,
         "cpu_baseline": cpu,

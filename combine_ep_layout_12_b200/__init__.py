@@ -76,7 +76,7 @@ class EPBuffer:
         self.recv_count = torch.empty((c.E, c.P), dtype=torch.int32, device=dev)
         self.dst_pos = torch.empty((c.B, c.k), dtype=torch.int32, device=dev)
         self.recv_src = torch.empty(self.rows, dtype=torch.int32, device=dev)
-        xdt = torch.int8 if c.quant_mode == 2 else torch.bfloat16
+        xdt = torch.int8 if c.quant_mode != 0 else torch.bfloat16
         self.recv_x = torch.empty((self.rows, c.d), dtype=xdt, device=dev)
         q = c.quant_mode == 2
         self.recv_scale = torch.empty(self.rows, dtype=torch.float32, device=dev) if q else None
@@ -97,30 +97,46 @@ class EPBuffer:
         except Exception:
             pass
 
+    def _mask(self, x_active_mask):
+        """x_active_mask: None or a [B] bool/uint8 device tensor (nonzero = active)."""
+        if x_active_mask is None:
+            return None
+        t = x_active_mask
+        if t.dtype not in (torch.bool, torch.uint8):
+            raise ValueError("x_active_mask must be bool or uint8, got %s" % t.dtype)
+        if tuple(t.shape) != (self.cfg.B,) or not t.is_contiguous() or t.device != self.device:
+            raise ValueError("x_active_mask must be a contiguous [B] tensor on %s" % self.device)
+        return _ptr(t)
+
+    def _smooth_shape(self):
+        c = self.cfg
+        return (c.d,) if c.smooth_rows <= 1 else (c.smooth_rows, c.d)
+
     # -- hot path ---------------------------------------------------------------
-    def layout(self, topk_idx, stream=None):
+    def layout(self, topk_idx, x_active_mask=None, stream=None):
         c = self.cfg
         _need(topk_idx, "topk_idx", torch.int32, (c.B, c.k), self.device)
-        ep_layout(self.handle, _ptr(topk_idx), _stream(stream))
+        ep_layout(self.handle, _ptr(topk_idx), self._mask(x_active_mask), _stream(stream))
 
     def dispatch(self, x, smooth_scale=None, stream=None):
         c = self.cfg
         _need(x, "x", torch.bfloat16, (c.B, c.d), self.device)
         if smooth_scale is not None:
-            _need(smooth_scale, "smooth_scale", torch.float32, (c.d,), self.device)
+            _need(smooth_scale, "smooth_scale", torch.float32, self._smooth_shape(), self.device)
         ep_dispatch(self.handle, _ptr(x), _ptr(smooth_scale), _stream(stream))
 
-    def layout_dispatch(self, topk_idx, x, smooth_scale=None, stream=None):
+    def layout_dispatch(self, topk_idx, x, smooth_scale=None, x_active_mask=None, stream=None):
         """layout(topk_idx) then dispatch(x), as one call (one grid when T <= 128)."""
         c = self.cfg
         _need(topk_idx, "topk_idx", torch.int32, (c.B, c.k), self.device)
         _need(x, "x", torch.bfloat16, (c.B, c.d), self.device)
         if smooth_scale is not None:
-            _need(smooth_scale, "smooth_scale", torch.float32, (c.d,), self.device)
-        ep_layout_dispatch(self.handle, _ptr(topk_idx), _ptr(x), _ptr(smooth_scale), _stream(stream))
+            _need(smooth_scale, "smooth_scale", torch.float32, self._smooth_shape(), self.device)
+        ep_layout_dispatch(self.handle, _ptr(topk_idx), self._mask(x_active_mask), _ptr(x),
+                           _ptr(smooth_scale), _stream(stream))
 
     def combine(self, expert_out, topk_idx, topk_weights, ori_x=None, a1=None, a2=None, v=None,
-                y=None, stream=None):
+                y=None, x_active_mask=None, stream=None):
         c = self.cfg
         _need(expert_out, "expert_out", torch.bfloat16, (self.rows, c.d), self.device)
         _need(topk_idx, "topk_idx", torch.int32, (c.B, c.k), self.device)
@@ -134,8 +150,9 @@ class EPBuffer:
             y = torch.empty((c.B, c.d), dtype=torch.bfloat16, device=self.device)
         else:
             _need(y, "y", torch.bfloat16, (c.B, c.d), self.device)
-        ep_combine(self.handle, _ptr(expert_out), _ptr(topk_idx), _ptr(topk_weights), _ptr(ori_x),
-                   _ptr(a1), _ptr(a2), _ptr(v), _ptr(y), _stream(stream))
+        ep_combine(self.handle, _ptr(expert_out), _ptr(topk_idx), _ptr(topk_weights),
+                   self._mask(x_active_mask), _ptr(ori_x), _ptr(a1), _ptr(a2), _ptr(v), _ptr(y),
+                   _stream(stream))
         return y
 
     def check(self, stream=None):

@@ -61,10 +61,10 @@ def lib():
     L.ep_buffer_create.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_buffer_ptrs),
                                    ctypes.POINTER(vp)]
     L.ep_buffer_destroy.argtypes = [vp]
-    L.ep_layout.argtypes = [vp, vp, vp]
+    L.ep_layout.argtypes = [vp, vp, vp, vp]
     L.ep_dispatch.argtypes = [vp, vp, vp, vp]
-    L.ep_layout_dispatch.argtypes = [vp, vp, vp, vp, vp]
-    L.ep_combine.argtypes = [vp] * 10
+    L.ep_layout_dispatch.argtypes = [vp] * 6
+    L.ep_combine.argtypes = [vp] * 11
     L.ep_buffer_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.ep_layout_static_scratch.argtypes = [ctypes.POINTER(ep_config)] + [vp] * 8
     for f in (L.ep_buffer_size, L.ep_buffer_create, L.ep_buffer_destroy, L.ep_layout,
@@ -108,22 +108,23 @@ def ep_buffer_destroy(handle):
     _check(lib().ep_buffer_destroy(handle), "ep_buffer_destroy")
 
 
-def ep_layout(handle, topk_idx, stream=0):
-    _check(lib().ep_layout(handle, topk_idx, stream), "ep_layout")
+def ep_layout(handle, topk_idx, x_active_mask=None, stream=0):
+    _check(lib().ep_layout(handle, topk_idx, x_active_mask, stream), "ep_layout")
 
 
 def ep_dispatch(handle, x, smooth_scale=None, stream=0):
     _check(lib().ep_dispatch(handle, x, smooth_scale, stream), "ep_dispatch")
 
 
-def ep_layout_dispatch(handle, topk_idx, x, smooth_scale=None, stream=0):
-    _check(lib().ep_layout_dispatch(handle, topk_idx, x, smooth_scale, stream),
+def ep_layout_dispatch(handle, topk_idx, x_active_mask, x, smooth_scale=None, stream=0):
+    _check(lib().ep_layout_dispatch(handle, topk_idx, x_active_mask, x, smooth_scale, stream),
            "ep_layout_dispatch")
 
 
-def ep_combine(handle, expert_out, topk_idx, topk_weights, ori_x, a1, a2, v, y, stream=0):
-    _check(lib().ep_combine(handle, expert_out, topk_idx, topk_weights, ori_x, a1, a2, v, y,
-                            stream), "ep_combine")
+def ep_combine(handle, expert_out, topk_idx, topk_weights, x_active_mask, ori_x, a1, a2, v, y,
+               stream=0):
+    _check(lib().ep_combine(handle, expert_out, topk_idx, topk_weights, x_active_mask, ori_x, a1,
+                            a2, v, y, stream), "ep_combine")
 
 
 def ep_buffer_check(handle, stream=0):

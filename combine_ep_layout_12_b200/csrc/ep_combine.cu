@@ -9,7 +9,8 @@
 //   e = fp32(expert_out[dst_pos[t][j]])          routed pick
 //       fp32(ori_x[t])                            copy expert
 //       a1[c]*ori_x[t] + a2[c]*v[c]  (fp32 ops)   constant expert c
-//   -1, zero experts, dropped picks: no term.
+//   -1, zero experts, dropped picks, every pick of an inactive token
+//   (x_active_mask): no term, so an inactive token gets y = +0.
 //
 // Design.  A CTA covers NT consecutive 16-byte column vectors (8 bf16) of one
 // token.  The token's k picks are classified once into shared memory, then each
@@ -30,6 +31,7 @@ constexpr int kCombineSelfRowsMaxT = 256;
 struct CombineArgs {
     const uint16_t* expert_out;  // [rows][d]
     const int32_t* topk_idx;     // [B][k]
+    const uint8_t* active;       // x_active_mask [B] or null: inactive tokens give +0
     const float* topk_weights;   // [B][k]
     const int32_t* dst_pos;      // [B][k]
     const uint16_t* ori_x;       // [B][d]
@@ -74,16 +76,17 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
     // y is written only after the wait.
     __shared__ int s_rows[KMAX], s_g[KMAX], s_cnt[KMAX];
     if (a.self_rows) {
-        routing_rows(a.topk_idx, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt);
+        routing_rows(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt);
     } else {
         pdl_wait();
     }
     pdl_launch_dependents();
 
     unsigned bad = 0;
+    const bool on = !(a.active && !a.active[t]);  // an inactive token has no terms
     if (threadIdx.x < a.k) {
         const size_t i = (size_t)t * a.k + threadIdx.x;
-        const int g = a.topk_idx[i];
+        const int g = on ? a.topk_idx[i] : -1;
         const int dp = a.self_rows ? s_rows[threadIdx.x] : a.dst_pos[i];
         int kind = kSkip;
         long long src = 0;
@@ -158,13 +161,15 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
 }  // namespace
 
 int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
-                   const int32_t* topk_idx, const float* topk_weights, const uint16_t* ori_x,
+                   const int32_t* topk_idx, const float* topk_weights, const uint8_t* active,
+                   const uint16_t* ori_x,
                    const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
                    cudaStream_t stream) {
     if (s.B == 0) return EP_OK;
     CombineArgs a;
     a.expert_out = expert_out;
     a.topk_idx = topk_idx;
+    a.active = active;
     a.topk_weights = topk_weights;
     a.dst_pos = p.dst_pos;
     a.ori_x = ori_x;

@@ -12,8 +12,10 @@ constexpr int kSelfRowsMaxT = 256;
 struct DispatchArgs {
     const uint16_t* x;       // [B][d] bf16
     const float* smooth;     // [d] or null
+    int expert_smooth;       // smooth holds one [d] row per routed expert (expert-major kernel)
     const int32_t* dst_pos;  // [B][k]
     const int32_t* topk_idx; // [B][k]; read instead of dst_pos when self_rows
+    const uint8_t* active;   // x_active_mask [B] or null (self_rows only: dst_pos has it)
     int self_rows;           // compute the receive rows here (small T) instead of reading dst_pos
     int T, P, M, E;
     void* recv_x;            // [rows][d] int8 or bf16
@@ -28,7 +30,7 @@ struct DispatchArgs {
 // while the x row load is in flight.
 __device__ __forceinline__ void compute_rows(const DispatchArgs& a, int t, int* s_rows, int* s_g,
                                              int* s_cnt) {
-    routing_rows(a.topk_idx, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt);
+    routing_rows(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt);
 }
 
 // Receive rows of token t into shared memory; out-of-range rows are skipped and flagged.
@@ -45,24 +47,46 @@ __device__ __forceinline__ void load_rows(const DispatchArgs& a, int t, int* s_r
     if (threadIdx.x < 32) report_err(a.err, bad);
 }
 
-// x_fp32 of the two bf16 halves of one 32-bit word, times the smooth scale when given.
-__device__ __forceinline__ void xf_pair(uint32_t w, const float* ss, int i, float& lo, float& hi) {
-    lo = bf16lo(w);
-    hi = bf16hi(w);
+// x_fp32 of one 16-element unit (two 16-byte bf16 vectors), times the smooth scale
+// when given (four 16-byte loads of it, kept in L1 for the second pass).
+__device__ __forceinline__ void xf_unit(const uint4 (&r)[2], const float* ss, float (&f)[16]) {
+    const uint32_t w[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        f[2 * e] = bf16lo(w[e]);
+        f[2 * e + 1] = bf16hi(w[e]);
+    }
     if (ss) {
-        lo = __fmul_rn(lo, ss[i]);
-        hi = __fmul_rn(hi, ss[i + 1]);
+        const float4* s4 = reinterpret_cast<const float4*>(ss);
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float4 m = __ldg(s4 + h);
+            f[4 * h] = __fmul_rn(f[4 * h], m.x);
+            f[4 * h + 1] = __fmul_rn(f[4 * h + 1], m.y);
+            f[4 * h + 2] = __fmul_rn(f[4 * h + 2], m.z);
+            f[4 * h + 3] = __fmul_rn(f[4 * h + 3], m.w);
+        }
     }
 }
 
-// CastToInt8 of x_fp32 * s: round half to even, saturate.
-__device__ __forceinline__ uint32_t q8(float xf, float s) {
-    const int q = min(127, max(-128, __float2int_rn(__fmul_rn(xf, s))));
-    return (uint32_t)(q & 0xff);
+// CastToInt8 of v, four at a time: round half to even, saturate, pack the bytes.
+// The clamp bounds are integers, so clamping before rounding equals saturating
+// after it.  The rounding itself is the classic magic-number conversion: adding
+// 1.5 * 2^23 in fp32 (round to nearest even) leaves rne(v) in the low mantissa
+// bits, exact for |v| < 2^22; the low byte of the sum is then q mod 256.  This is
+// one add and a byte permute per value instead of a float-to-int conversion.
+__device__ __forceinline__ uint32_t s8_byte_word(float v) {
+    return __float_as_uint(__fadd_rn(fminf(fmaxf(v, -128.0f), 127.0f), 12582912.0f));
+}
+__device__ __forceinline__ uint32_t cvt_s8x4(float a, float b, float c, float d) {
+    const uint32_t lo = __byte_perm(s8_byte_word(a), s8_byte_word(b), 0x0040);
+    const uint32_t hi = __byte_perm(s8_byte_word(c), s8_byte_word(d), 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
 }
 
-// quant_mode 2: a unit is 16 elements (two 16-byte bf16 loads -> one 16-byte int8 store).
-template <int U>
+// quant_mode 2 (dynamic) or 1 (STATIC: q = CastToInt8(x_fp32), no absmax and no
+// scale): a unit is 16 elements (two 16-byte bf16 loads -> one 16-byte int8 store).
+template <int U, bool STATIC>
 __device__ __forceinline__ void dispatch_int8_body(const DispatchArgs& a, int t) {
     __shared__ int s_rows[kMaxK];
     __shared__ float s_red[32];
@@ -89,62 +113,59 @@ __device__ __forceinline__ void dispatch_int8_body(const DispatchArgs& a, int t)
     else
         load_rows(a, t, s_rows);
 
-    // x_fp32 = fp32(x) * smooth; absmax over the row
-    float amax = 0.0f;
+    float s = 1.0f, inv = 0.0f;
+    bool degenerate = false;
+    if (STATIC) {
+        __syncthreads();  // publishes s_rows
+    } else {
+        // x_fp32 = fp32(x) * smooth; absmax over the row
+        float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < U; ++i) {
-        const int u = threadIdx.x + i * NT;
-        if (u >= nunits) continue;
-        const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
-                               raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
-        const float* ss = a.smooth ? a.smooth + 16 * u : nullptr;
+        for (int i = 0; i < U; ++i) {
+            const int u = threadIdx.x + i * NT;
+            if (u >= nunits) continue;
+            float f[16];
+            xf_unit(raw[i], a.smooth ? a.smooth + 16 * u : nullptr, f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            float lo, hi;
-            xf_pair(w[e], ss, 2 * e, lo, hi);
-            amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
         }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
-    __syncthreads();  // also publishes s_rows
-    if (threadIdx.x < 32) {
-        float m = threadIdx.x < (NT >> 5) ? s_red[threadIdx.x] : 0.0f;
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = amax;
+        __syncthreads();  // also publishes s_rows
+        if (threadIdx.x < 32) {
+            float m = threadIdx.x < (NT >> 5) ? s_red[threadIdx.x] : 0.0f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (threadIdx.x == 0) s_red[0] = m;
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if (threadIdx.x == 0) s_red[0] = m;
+        }
+        __syncthreads();
+        amax = s_red[0];
+        s = __fdiv_rn(127.0f, amax);
+        degenerate = (amax == 0.0f) || isinf(s);
+        inv = degenerate ? 0.0f : __fdiv_rn(1.0f, s);
     }
-    __syncthreads();
-    amax = s_red[0];
-
-    const float s = __fdiv_rn(127.0f, amax);
-    const bool degenerate = (amax == 0.0f) || isinf(s);
-    const float inv = degenerate ? 0.0f : __fdiv_rn(1.0f, s);
     int8_t* out = reinterpret_cast<int8_t*>(a.recv_x);
 
 #pragma unroll
     for (int i = 0; i < U; ++i) {
         const int u = threadIdx.x + i * NT;
         if (u >= nunits) continue;
-        const uint32_t w[8] = {raw[i][0].x, raw[i][0].y, raw[i][0].z, raw[i][0].w,
-                               raw[i][1].x, raw[i][1].y, raw[i][1].z, raw[i][1].w};
-        const float* ss = a.smooth ? a.smooth + 16 * u : nullptr;
-        uint32_t word[4];
+        float f[16];
+        xf_unit(raw[i], a.smooth ? a.smooth + 16 * u : nullptr, f);
+        if (!STATIC) {
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            float x0, x1, x2, x3;
-            xf_pair(w[2 * h], ss, 4 * h, x0, x1);
-            xf_pair(w[2 * h + 1], ss, 4 * h + 2, x2, x3);
-            word[h] = degenerate ? 0u
-                                 : (q8(x0, s) | (q8(x1, s) << 8) | (q8(x2, s) << 16) | (q8(x3, s) << 24));
+            for (int e = 0; e < 16; ++e) f[e] = __fmul_rn(f[e], s);
         }
-        const uint4 v = make_uint4(word[0], word[1], word[2], word[3]);
+        uint4 v = make_uint4(cvt_s8x4(f[0], f[1], f[2], f[3]), cvt_s8x4(f[4], f[5], f[6], f[7]),
+                             cvt_s8x4(f[8], f[9], f[10], f[11]), cvt_s8x4(f[12], f[13], f[14], f[15]));
+        if (degenerate) v = make_uint4(0, 0, 0, 0);
         for (int j = 0; j < a.k; ++j) {
             const int row = s_rows[j];
             if (row >= 0) st_v4(out + (size_t)row * a.d + 16 * u, v);
         }
     }
+    if (STATIC) return;
     if (threadIdx.x < a.k) {
         const int row = s_rows[threadIdx.x];
         if (row >= 0) a.recv_scale[row] = inv;
@@ -187,10 +208,13 @@ __device__ __forceinline__ void dispatch_bf16_body(const DispatchArgs& a, int t)
 
 // Host-side helpers shared by the dispatch launchers.
 inline DispatchArgs make_dispatch_args(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
-                                       const float* smooth, const int32_t* topk_idx) {
+                                       const float* smooth, const int32_t* topk_idx,
+                                       const uint8_t* active) {
     DispatchArgs a;
+    a.active = active;
     a.x = x;
     a.smooth = smooth;
+    a.expert_smooth = (smooth != nullptr && s.expert_smooth) ? 1 : 0;
     a.dst_pos = p.dst_pos;
     a.recv_x = p.recv_x;
     a.recv_scale = p.recv_scale;

@@ -14,7 +14,8 @@
 namespace ep {
 namespace {
 
-template <int KM, int U, bool INT8>
+// MODE: quant_mode (0 bf16 pass-through, 1 static int8, 2 dynamic int8).
+template <int KM, int U, int MODE>
 __global__ void __launch_bounds__(128, (U <= 4 ? 8 : 4))
     layout_dispatch_kernel(LayoutArgs la, DispatchArgs da, int cpr, int n_layout) {
     extern __shared__ unsigned smem[];
@@ -22,37 +23,47 @@ __global__ void __launch_bounds__(128, (U <= 4 ? 8 : 4))
     pdl_launch_dependents();
     if ((int)blockIdx.x < n_layout) {
         layout_small_body<KM>(la, cpr, blockIdx.x, smem);
-    } else if (INT8) {
-        dispatch_int8_body<U>(da, blockIdx.x - n_layout);
-    } else {
+    } else if (MODE == 0) {
         dispatch_bf16_body<U>(da, blockIdx.x - n_layout);
+    } else {
+        dispatch_int8_body<U, MODE == 1>(da, blockIdx.x - n_layout);
     }
 }
 
-template <int KM, bool INT8>
+template <int KM, int MODE>
 cudaError_t launch_fused_u(int U, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                            const LayoutArgs& la, const DispatchArgs& da, int cpr, int n_layout) {
     switch (U) {
-        case 1: return launch_pdl(layout_dispatch_kernel<KM, 1, INT8>, grid, block, smem, stream, la, da, cpr, n_layout);
-        case 2: return launch_pdl(layout_dispatch_kernel<KM, 2, INT8>, grid, block, smem, stream, la, da, cpr, n_layout);
-        case 4: return launch_pdl(layout_dispatch_kernel<KM, 4, INT8>, grid, block, smem, stream, la, da, cpr, n_layout);
-        default: return launch_pdl(layout_dispatch_kernel<KM, 8, INT8>, grid, block, smem, stream, la, da, cpr, n_layout);
+        case 1: return launch_pdl(layout_dispatch_kernel<KM, 1, MODE>, grid, block, smem, stream, la, da, cpr, n_layout);
+        case 2: return launch_pdl(layout_dispatch_kernel<KM, 2, MODE>, grid, block, smem, stream, la, da, cpr, n_layout);
+        case 4: return launch_pdl(layout_dispatch_kernel<KM, 4, MODE>, grid, block, smem, stream, la, da, cpr, n_layout);
+        default: return launch_pdl(layout_dispatch_kernel<KM, 8, MODE>, grid, block, smem, stream, la, da, cpr, n_layout);
     }
+}
+
+template <int KM>
+cudaError_t launch_fused_mode(int mode, int U, dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              const LayoutArgs& la, const DispatchArgs& da, int cpr, int n_layout) {
+    if (mode == 0) return launch_fused_u<KM, 0>(U, grid, block, smem, stream, la, da, cpr, n_layout);
+    if (mode == 1) return launch_fused_u<KM, 1>(U, grid, block, smem, stream, la, da, cpr, n_layout);
+    return launch_fused_u<KM, 2>(U, grid, block, smem, stream, la, da, cpr, n_layout);
 }
 
 }  // namespace
 
 int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
-                           const uint16_t* x, const float* smooth, cudaStream_t stream) {
+                           const uint8_t* active, const uint16_t* x, const float* smooth,
+                           cudaStream_t stream) {
     const int cpr = (s.T + 31) / 32;
     int U = 0, NT = 0;
-    const int units = s.quant_mode == 2 ? s.d / 16 : s.d / 8;
+    const int units = s.quant_mode != 0 ? s.d / 16 : s.d / 8;
     const bool fits = s.B > 0 && s.layout == 0 && cpr <= 4 && s.k <= 8 &&
+                      !(smooth && s.expert_smooth) &&
                       pick_units(units, 8, &U, &NT) == EP_OK &&
                       NT <= 128 && U <= 8;
     if (!fits) {
-        const int st = launch_layout(s, p, topk_idx, stream);
-        return st != EP_OK ? st : launch_dispatch(s, p, x, smooth, topk_idx, stream);
+        const int st = launch_layout(s, p, topk_idx, active, stream);
+        return st != EP_OK ? st : launch_dispatch(s, p, x, smooth, topk_idx, active, stream);
     }
     const int threads = NT > 32 * cpr ? NT : 32 * cpr;  // the layout part needs one warp per chunk
     const int warps = threads / 32;
@@ -64,6 +75,7 @@ int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_
 
     LayoutArgs la;
     la.topk_idx = topk_idx;
+    la.active = active;
     la.expert_count = p.expert_count;
     la.expert_offset = p.expert_offset;
     la.recv_count = p.recv_count;
@@ -74,21 +86,17 @@ int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_
     la.B = s.B; la.k = s.k; la.P = s.P; la.M = s.M; la.E = s.E; la.T = s.T;
     la.n_special = s.n_special; la.E_tot = s.E_tot;
     la.warps = warps;
-    DispatchArgs da = make_dispatch_args(s, p, x, smooth, topk_idx);
+    DispatchArgs da = make_dispatch_args(s, p, x, smooth, topk_idx, active);
     da.self_rows = 1;
 
     const dim3 grid((unsigned)(n_layout + s.B)), block((unsigned)threads);
     cudaError_t e;
-    const bool int8 = s.quant_mode == 2;
     if (s.k <= 2)
-        e = int8 ? launch_fused_u<2, true>(U, grid, block, smem, stream, la, da, cpr, n_layout)
-                 : launch_fused_u<2, false>(U, grid, block, smem, stream, la, da, cpr, n_layout);
+        e = launch_fused_mode<2>(s.quant_mode, U, grid, block, smem, stream, la, da, cpr, n_layout);
     else if (s.k <= 4)
-        e = int8 ? launch_fused_u<4, true>(U, grid, block, smem, stream, la, da, cpr, n_layout)
-                 : launch_fused_u<4, false>(U, grid, block, smem, stream, la, da, cpr, n_layout);
+        e = launch_fused_mode<4>(s.quant_mode, U, grid, block, smem, stream, la, da, cpr, n_layout);
     else
-        e = int8 ? launch_fused_u<8, true>(U, grid, block, smem, stream, la, da, cpr, n_layout)
-                 : launch_fused_u<8, false>(U, grid, block, smem, stream, la, da, cpr, n_layout);
+        e = launch_fused_mode<8>(s.quant_mode, U, grid, block, smem, stream, la, da, cpr, n_layout);
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 

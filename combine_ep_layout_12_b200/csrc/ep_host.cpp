@@ -15,6 +15,7 @@ struct ep_buffer {
     ep_buffer_ptrs ptrs;
     ep_buffer_sizes sizes;
     const int32_t* last_topk_idx;  // routing of the latest ep_layout (dispatch may re-read it)
+    const uint8_t* last_active;    // its x_active_mask (or null)
 };
 
 namespace {
@@ -28,8 +29,9 @@ int check_config(const ep_config* c) {
         return EP_ERR_INVALID_ARG;
     if (c->n_zero < 0 || c->n_copy < 0 || c->n_const < 0) return EP_ERR_INVALID_ARG;
     if (c->B % c->P != 0 || c->E % c->P != 0) return EP_ERR_INVALID_ARG;
-    if (c->quant_mode != 0 && c->quant_mode != 2) return EP_ERR_INVALID_ARG;
-    if (c->smooth_rows != 0 && c->smooth_rows != 1) return EP_ERR_INVALID_ARG;
+    if (c->quant_mode < 0 || c->quant_mode > 2) return EP_ERR_INVALID_ARG;
+    if (c->smooth_rows != 0 && c->smooth_rows != 1 && c->smooth_rows != c->E) return EP_ERR_INVALID_ARG;
+    if (c->smooth_rows > 1 && c->quant_mode == 0) return EP_ERR_INVALID_ARG;
     if (c->layout != 0 && c->layout != 1) return EP_ERR_UNSUPPORTED;
     if (c->d % 16 != 0) return EP_ERR_INVALID_ARG;
     if (c->k > ep::kMaxK) return EP_ERR_INVALID_ARG;
@@ -53,7 +55,7 @@ void fill_sizes(const ep_config* c, ep_buffer_sizes* s) {
     const size_t E_tot = (size_t)c->E + c->n_zero + c->n_copy + c->n_const;
     const size_t n_special = (size_t)c->n_zero + c->n_copy + c->n_const;
     const size_t rows = (size_t)ep::make_shape(*c).rows;
-    const size_t esz = c->quant_mode == 2 ? 1 : 2;
+    const size_t esz = c->quant_mode != 0 ? 1 : 2;
     s->expert_count = 4 * E_tot;
     s->expert_offset = 4 * (E_tot + 1);
     s->recv_count = 4 * (size_t)c->E * c->P;
@@ -101,6 +103,7 @@ int ep_buffer_create(const ep_config* cfg, const ep_buffer_ptrs* ptrs, ep_buffer
     b->ptrs = *ptrs;
     b->sizes = s;
     b->last_topk_idx = nullptr;
+    b->last_active = nullptr;
     *out = b;
     return EP_OK;
 }
@@ -110,12 +113,14 @@ int ep_buffer_destroy(ep_buffer* buf) {
     return EP_OK;
 }
 
-int ep_layout(ep_buffer* buf, const int32_t* topk_idx, ep_stream_t stream) {
+int ep_layout(ep_buffer* buf, const int32_t* topk_idx, const uint8_t* x_active_mask,
+              ep_stream_t stream) {
     if (!buf) return EP_ERR_INVALID_ARG;
     if (buf->cfg.B > 0 && (!topk_idx || !aligned4(topk_idx))) return EP_ERR_INVALID_ARG;
-    const int st = ep::launch_layout(ep::make_shape(buf->cfg), buf->ptrs, topk_idx,
+    const int st = ep::launch_layout(ep::make_shape(buf->cfg), buf->ptrs, topk_idx, x_active_mask,
                                      reinterpret_cast<cudaStream_t>(stream));
     buf->last_topk_idx = st == EP_OK ? topk_idx : nullptr;
+    buf->last_active = st == EP_OK ? x_active_mask : nullptr;
     return st;
 }
 
@@ -124,28 +129,31 @@ int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale, ep
     const ep_config& c = buf->cfg;
     if (c.B > 0 && (!x || !aligned16(x))) return EP_ERR_INVALID_ARG;
     if (smooth_scale && (c.smooth_rows == 0 || !aligned16(smooth_scale))) return EP_ERR_INVALID_ARG;
-    if (smooth_scale && c.quant_mode != 2) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && c.quant_mode == 0) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && c.smooth_rows > 1 && c.B > 0 && !buf->last_topk_idx) return EP_ERR_INVALID_ARG;
     return ep::launch_dispatch(ep::make_shape(c), buf->ptrs, x, smooth_scale, buf->last_topk_idx,
-                               reinterpret_cast<cudaStream_t>(stream));
+                               buf->last_active, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx, const uint16_t* x,
-                       const float* smooth_scale, ep_stream_t stream) {
+int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx, const uint8_t* x_active_mask,
+                       const uint16_t* x, const float* smooth_scale, ep_stream_t stream) {
     if (!buf) return EP_ERR_INVALID_ARG;
     const ep_config& c = buf->cfg;
     if (c.B > 0 && (!topk_idx || !aligned4(topk_idx))) return EP_ERR_INVALID_ARG;
     if (c.B > 0 && (!x || !aligned16(x))) return EP_ERR_INVALID_ARG;
     if (smooth_scale && (c.smooth_rows == 0 || !aligned16(smooth_scale))) return EP_ERR_INVALID_ARG;
-    if (smooth_scale && c.quant_mode != 2) return EP_ERR_INVALID_ARG;
-    const int st = ep::launch_layout_dispatch(ep::make_shape(c), buf->ptrs, topk_idx, x, smooth_scale,
-                                              reinterpret_cast<cudaStream_t>(stream));
+    if (smooth_scale && c.quant_mode == 0) return EP_ERR_INVALID_ARG;
+    const int st = ep::launch_layout_dispatch(ep::make_shape(c), buf->ptrs, topk_idx, x_active_mask,
+                                              x, smooth_scale, reinterpret_cast<cudaStream_t>(stream));
     buf->last_topk_idx = st == EP_OK ? topk_idx : nullptr;
+    buf->last_active = st == EP_OK ? x_active_mask : nullptr;
     return st;
 }
 
 int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,
-               const float* topk_weights, const uint16_t* ori_x, const uint16_t* a1,
-               const uint16_t* a2, const uint16_t* v, uint16_t* y, ep_stream_t stream) {
+               const float* topk_weights, const uint8_t* x_active_mask, const uint16_t* ori_x,
+               const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
+               ep_stream_t stream) {
     if (!buf) return EP_ERR_INVALID_ARG;
     const ep_config& c = buf->cfg;
     if (c.B > 0) {
@@ -159,7 +167,8 @@ int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_i
         if (y == ori_x || y == expert_out) return EP_ERR_INVALID_ARG;
     }
     return ep::launch_combine(ep::make_shape(c), buf->ptrs, expert_out, topk_idx, topk_weights,
-                              ori_x, a1, a2, v, y, reinterpret_cast<cudaStream_t>(stream));
+                              x_active_mask, ori_x, a1, a2, v, y,
+                              reinterpret_cast<cudaStream_t>(stream));
 }
 
 int ep_buffer_check(ep_buffer* buf, ep_stream_t stream, uint32_t* err_bits) {

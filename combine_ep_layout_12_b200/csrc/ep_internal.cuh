@@ -27,7 +27,8 @@ constexpr int kMaxPackedEP = 24576;  // E * P of the packed layout (the pack ker
 
 struct Shape {
     int B, d, k, P, M, E, Z, C, K, T, L, E_tot, n_special;
-    int quant_mode;
+    int quant_mode;     // 0 bf16, 1 static int8, 2 dynamic int8
+    int expert_smooth;  // 1: a given smooth scale is [E][d], one row per routed expert
     int layout;      // 0 low-latency, 1 packed
     long long rows;  // receive rows: E * P * M (low-latency) or B * k (packed)
 };
@@ -41,6 +42,7 @@ inline Shape make_shape(const ep_config& c) {
     s.n_special = c.n_zero + c.n_copy + c.n_const;
     s.E_tot = c.E + s.n_special;
     s.quant_mode = c.quant_mode;
+    s.expert_smooth = c.smooth_rows > 1 ? 1 : 0;
     s.layout = c.layout;
     s.rows = c.layout == 1 ? (long long)c.B * c.k : (long long)c.E * c.P * c.M;
     return s;
@@ -56,18 +58,24 @@ inline size_t workspace_bytes(const Shape& s) {
 }
 
 // Host launchers (one per kernel family); each returns an EP_* status.
+// active: x_active_mask [B] (nonzero = active) or null; an inactive token takes no
+// part (as if every pick were -1).
 int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
-                  cudaStream_t stream);
+                  const uint8_t* active, cudaStream_t stream);
 // topk_idx: the routing of the latest layout on this buffer (lets dispatch derive
-// its receive rows itself for small per-rank batches); may be null.
+// its receive rows itself for small per-rank batches); may be null, except with a
+// per-expert smooth scale, where it names each copy's expert.
 int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
-                    const float* smooth, const int32_t* topk_idx, cudaStream_t stream);
+                    const float* smooth, const int32_t* topk_idx, const uint8_t* active,
+                    cudaStream_t stream);
 // Layout and dispatch of the same routing in one grid when the batch per rank is
 // small (T <= 128, k <= 8); otherwise the two launches above, in order.
 int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
-                           const uint16_t* x, const float* smooth, cudaStream_t stream);
+                           const uint8_t* active, const uint16_t* x, const float* smooth,
+                           cudaStream_t stream);
 int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
-                   const int32_t* topk_idx, const float* topk_weights, const uint16_t* ori_x,
+                   const int32_t* topk_idx, const float* topk_weights, const uint8_t* active,
+                   const uint16_t* ori_x,
                    const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
                    cudaStream_t stream);
 
@@ -163,15 +171,16 @@ __device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
 // batches: the slot of a routed id g is the number of earlier tokens of the same
 // rank that picked g (a token counts once), which is exactly the slot the layout
 // kernels assign; a routed id repeated inside the token gets row -1 after its
-// first occurrence.  The earlier tokens' ids come from L2.  s_rows, s_g, s_cnt:
-// k-entry shared arrays.  All threads of the CTA call it; on return s_rows[j] is
-// written by thread j (j < k) and not yet published to the other threads.
-__device__ inline void routing_rows(const int32_t* topk_idx, int t, int k, int E, int T, int P,
-                                    int M, int* s_rows, int* s_g, int* s_cnt) {
+// first occurrence.  Inactive tokens (active[t] == 0, when a mask is given) route
+// nothing and are not counted.  The earlier tokens' ids come from L2.  s_rows,
+// s_g, s_cnt: k-entry shared arrays.  All threads of the CTA call it; on return
+// s_rows[j] is written by thread j (j < k) and not yet published to the other threads.
+__device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* active, int t, int k,
+                                    int E, int T, int P, int M, int* s_rows, int* s_g, int* s_cnt) {
     if (threadIdx.x < k) {
         const int j = threadIdx.x;
         const int g = topk_idx[(size_t)t * k + j];
-        bool routed = g >= 0 && g < E;
+        bool routed = g >= 0 && g < E && !(active && !active[t]);
         for (int jj = 0; jj < j; ++jj)
             if (topk_idx[(size_t)t * k + jj] == g) routed = false;  // repeated id: dropped
         s_g[j] = routed ? g : -1;
@@ -180,6 +189,7 @@ __device__ inline void routing_rows(const int32_t* topk_idx, int t, int k, int E
     __syncthreads();
     const int r = t / T;
     for (int tt = r * T + (int)threadIdx.x; tt < t; tt += blockDim.x) {
+        if (active && !active[tt]) continue;
         const int32_t* ids = topk_idx + (size_t)tt * k;
         unsigned hit = 0;
         for (int jj = 0; jj < k; ++jj) {

@@ -73,11 +73,12 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
         const bool valid = t < tok_end;
         int ids[KM];
         bool routed[KM];
+        const bool on = valid && !(a.active && !a.active[t]);  // x_active_mask
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
             ids[j] = -1;
             routed[j] = false;
-            if (j < k && valid) ids[j] = a.topk_idx[(size_t)t * k + j];
+            if (j < k && on) ids[j] = a.topk_idx[(size_t)t * k + j];
         }
         // (2) classify; routed ids set their lane bit
 #pragma unroll
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(256) layout_pack_kernel(const int32_t* expert_
 }  // namespace
 
 int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
-                  cudaStream_t stream) {
+                  const uint8_t* active, cudaStream_t stream) {
     if (s.layout == 1 && s.B > 0) {
         // counts and low-latency-form rows (stride T, no recv_src), then pack
         Shape ll = s;
@@ -221,7 +222,7 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         ll.rows = (long long)s.E * s.P * s.T;
         ep_buffer_ptrs q = p;
         q.recv_src = nullptr;
-        const int st = launch_layout(ll, q, topk_idx, stream);
+        const int st = launch_layout(ll, q, topk_idx, active, stream);
         if (st != EP_OK) return st;
         const size_t smem = sizeof(int) * (size_t)s.E * s.P;
         static bool attr_pack[64] = {false};
@@ -268,6 +269,7 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         }
         LayoutArgs a1;
         a1.topk_idx = topk_idx;
+        a1.active = active;
         a1.expert_count = p.expert_count;
         a1.expert_offset = p.expert_offset;
         a1.recv_count = p.recv_count;
@@ -318,6 +320,7 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
 
     LayoutArgs a;
     a.topk_idx = topk_idx;
+    a.active = active;
     a.expert_count = p.expert_count;
     a.expert_offset = p.expert_offset;
     a.recv_count = p.recv_count;
@@ -412,7 +415,7 @@ extern "C" int ep_layout_static_scratch(const ep_config* cfg, const int32_t* top
     p.dst_pos = dst_pos;
     p.recv_src = recv_src;
     p.workspace = scratch;
-    const int lst = ep::launch_layout(ep::make_shape(*cfg), p, topk_idx, s);
+    const int lst = ep::launch_layout(ep::make_shape(*cfg), p, topk_idx, nullptr, s);
     if (lst != EP_OK) return lst;
     if (err_word) {
         const auto* hdr = reinterpret_cast<const ep::WsHeader*>(scratch);

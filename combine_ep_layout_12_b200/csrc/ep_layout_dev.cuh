@@ -9,6 +9,7 @@ namespace {
 
 struct LayoutArgs {
     const int32_t* topk_idx;
+    const uint8_t* active;  // x_active_mask [B] or null
     int32_t* expert_count;
     int32_t* expert_offset;
     int32_t* recv_count;
@@ -79,6 +80,15 @@ __device__ __forceinline__ void load_token_ids(const int32_t* topk_idx, int t, i
     }
 }
 
+// An inactive token (x_active_mask entry 0) is seen as k picks of -1.
+template <int KM>
+__device__ __forceinline__ void apply_active(const uint8_t* active, int t, int* ids) {
+    if (active && !active[t]) {
+#pragma unroll
+        for (int j = 0; j < KM; ++j) ids[j] = -1;
+    }
+}
+
 // Classify the picks of one token: returns a mask with bit j set when pick j is
 // routed (the first occurrence of an id in [0, E)); repeated routed ids and ids
 // outside [-1, E_tot) set error bits; specials are handed to on_special.
@@ -145,6 +155,7 @@ __device__ __forceinline__ void layout_small_body(const LayoutArgs& a, int cpr, 
                 const int t = t0 + b * stride;
                 if (t < a.B) {
                     load_token_ids<KM>(a.topk_idx, t, k, vec4, ids[b]);
+                    apply_active<KM>(a.active, t, ids[b]);
                 } else {
 #pragma unroll
                     for (int j = 0; j < KM; ++j) ids[b][j] = -1;
@@ -172,17 +183,18 @@ __device__ __forceinline__ void layout_small_body(const LayoutArgs& a, int cpr, 
     const int ranks_per_cta = (int)(blockDim.x >> 5) / cpr;
     const int lr = warp / cpr, c = warp - lr * cpr;
     const int r = (cta - 1) * ranks_per_cta + lr;
-    const bool active = lr < ranks_per_cta && r < P;
+    const bool holds_rank = lr < ranks_per_cta && r < P;
     unsigned* mask = reinterpret_cast<unsigned*>(smem);  // [warps][E]
     unsigned* my_mask = mask + (size_t)warp * E;
     for (int g = lane; g < E; g += 32) my_mask[g] = 0u;
     __syncthreads();
     const int t = a.T * r + c * 32 + lane;
-    const bool valid = active && c * 32 + lane < a.T;
+    const bool valid = holds_rank && c * 32 + lane < a.T;
     int ids[KM];
     unsigned rb = 0;
     if (valid) {
         load_token_ids<KM>(a.topk_idx, t, k, vec4, ids);
+        apply_active<KM>(a.active, t, ids);
         rb = classify_ids<KM>(ids, k, E, a.E_tot, err, [](int) {});
     }
 #pragma unroll

@@ -31,7 +31,7 @@ def to_device(inp, device, pin=False):
         else:
             out[name] = bf16_tensor(a, device)
     for name, dt in (("topk_idx", torch.int32), ("topk_weights", torch.float32),
-                     ("smooth", torch.float32)):
+                     ("smooth", torch.float32), ("active", torch.uint8)):
         a = inp.get(name)
         if a is None:
             out[name] = None
@@ -63,7 +63,7 @@ class Pipeline:
         self.y = torch.empty((w.B, w.d), dtype=torch.bfloat16, device=self.device)
 
     def layout(self, dev_inp, stream=None):
-        self.buf.layout(dev_inp["topk_idx"], stream=stream)
+        self.buf.layout(dev_inp["topk_idx"], x_active_mask=dev_inp.get("active"), stream=stream)
 
     def dispatch(self, dev_inp, stream=None):
         self.buf.dispatch(dev_inp["x"], dev_inp.get("smooth"), stream=stream)
@@ -71,11 +71,12 @@ class Pipeline:
     def combine(self, dev_inp, stream=None):
         return self.buf.combine(self.expert_out, dev_inp["topk_idx"], dev_inp["topk_weights"],
                                 ori_x=dev_inp["x"], a1=dev_inp.get("a1"), a2=dev_inp.get("a2"),
-                                v=dev_inp.get("v"), y=self.y, stream=stream)
+                                v=dev_inp.get("v"), y=self.y, x_active_mask=dev_inp.get("active"),
+                                stream=stream)
 
     def layout_dispatch(self, dev_inp, stream=None):
         self.buf.layout_dispatch(dev_inp["topk_idx"], dev_inp["x"], dev_inp.get("smooth"),
-                                 stream=stream)
+                                 x_active_mask=dev_inp.get("active"), stream=stream)
 
     def step(self, dev_inp, stream=None, fused=True):
         """layout -> dispatch -> combine; fused=True issues the first two as one call."""

@@ -14,7 +14,10 @@ Recipe (all from numpy.random.default_rng streams spawned from one seed):
               draw order; expert 0 is the hottest.
   weights     softmax (fp64, cast to fp32) of N(0, 1) logits, [B, k]
   a1, a2      U(0, 1) per element, [n_const, d] bf16;  v  N(0, 1), [n_const, d] bf16
-  smooth      "none" (absent), "ones" ([d] of 1.0) or "rand" (U(0.5, 2) per channel)
+  smooth      "none" (absent), "ones" ([d] of 1.0), "rand" (U(0.5, 2) per channel) or
+              "expert" (U(0.5, 2) per expert and channel, [E, d])
+  active      x_active_mask: absent when active_frac is None, else uint8 [B] with
+              each token active with probability active_frac
 """
 from dataclasses import dataclass, replace
 
@@ -40,6 +43,7 @@ class Workload:
     smooth: str = "none"
     seed: int = 0
     layout: int = 0  # 0: low-latency receive rows [E][P*M]; 1: packed rows [B*k]
+    active_frac: float = None  # x_active_mask: None = no mask
 
     @property
     def T(self):
@@ -52,6 +56,11 @@ class Workload:
     @property
     def E_tot(self):
         return self.E + self.n_zero + self.n_copy + self.n_const
+
+    @property
+    def smooth_rows(self):
+        """Rows of the smooth scale: E for a per-expert scale, else 1."""
+        return self.E if self.smooth == "expert" else 1
 
     @property
     def rows(self):
@@ -83,6 +92,17 @@ WORKLOADS = {
     "skewed": Workload("skewed", B=8192, d=4096, k=6, P=8, M=1024, E=64, n_zero=1, n_copy=1,
                        n_const=1, quant_mode=2, routing="zipf", zipf_s=1.2),
 }
+# per-expert smooth scale [E, d] (one quantization per routed copy), decode shape
+WORKLOADS["decode_expert_smooth"] = replace(WORKLOADS["decode"], name="decode_expert_smooth",
+                                            smooth="expert")
+# the same on the 64-expert receive buffer (1.4 GB), for multi-pass profiler captures
+WORKLOADS["decode_e64_expert_smooth"] = replace(WORKLOADS["decode_e64"], name="decode_e64_expert_smooth",
+                                                smooth="expert")
+# static int8 (quant_mode 1) with a [d] scale, decode shape
+WORKLOADS["decode_static"] = replace(WORKLOADS["decode"], name="decode_static", quant_mode=1,
+                                     smooth="rand")
+# decode with an x_active_mask of 3/4 of the tokens active
+WORKLOADS["decode_active"] = replace(WORKLOADS["decode"], name="decode_active", active_frac=0.75)
 SWEEP_T = (1, 4, 16, 64, 256, 1024, 4096)
 for _T in SWEEP_T:
     for _qm in (0, 2):
@@ -107,7 +127,7 @@ def f32_to_bf16_bits(a):
 
 def _streams(seed):
     ss = np.random.SeedSequence(seed)
-    names = ("x", "idx", "w", "const", "smooth", "expert")
+    names = ("x", "idx", "w", "const", "smooth", "expert", "active")
     return {n: np.random.default_rng(s) for n, s in zip(names, ss.spawn(len(names)))}
 
 
@@ -170,8 +190,14 @@ def generate(w: Workload, with_x=True):
         inp["smooth"] = np.ones(w.d, np.float32)
     elif w.smooth == "rand":
         inp["smooth"] = rs["smooth"].uniform(0.5, 2.0, w.d).astype(np.float32)
+    elif w.smooth == "expert":
+        inp["smooth"] = rs["smooth"].uniform(0.5, 2.0, (w.E, w.d)).astype(np.float32)
     else:
         raise ValueError(w.smooth)
+    if w.active_frac is None:
+        inp["active"] = None
+    else:
+        inp["active"] = (rs["active"].random(w.B) < w.active_frac).astype(np.uint8)
     return inp
 
 

@@ -25,11 +25,26 @@
  *               routed to g, ascending t (the page states the computation is
  *               deterministic).
  *   ep_dispatch quant_mode 0: expand_x row = x[t] (bf16 bits copied).
+ *               quant_mode 1 (static; the Formula's non-dynamic case with a mode
+ *               other than 0): q = CastToInt8(fp32(x) * smooth_scale) (round half
+ *               to even, saturate; no smooth scale = no multiply), no scale sent.
  *               quant_mode 2: xf = fp32(x) * smooth_scale, s = 127 / max|xf| over
  *               the row, q = CastToInt8(xf * s) (round half to even, saturate),
  *               inv = 1 / s; q goes to every receive row of t and inv to
  *               recv_scale of those rows and to token_scale[t]
- *               (Ascend Formula, dynamic quantization scenario).
+ *               (Ascend Formula, dynamic quantization scenario).  With a
+ *               per-expert smooth scale ([E][d], the scales of shape
+ *               [num_experts, h] in the Ascend Example) each routed copy (t, g)
+ *               is quantized on its own with xf = fp32(x) * smooth_scale[g]: its
+ *               own absmax, q and inv (in recv_scale of its row); token_scale is
+ *               then not written.  In quant_mode 1 a per-expert scale gives each
+ *               copy CastToInt8(fp32(x) * smooth_scale[g]).
+ *   x_active_mask (Ascend Prototype: the optional x_active_mask of
+ *               low_latency_dispatch; uint8 [B], nonzero = active, NULL = all
+ *               active): an inactive token takes no part, exactly as if each of
+ *               its picks were -1: no receive row, not counted in any count
+ *               (special experts included), no error bit for its ids, and combine
+ *               writes y[t] = +0.  In quant_mode 2 its token_scale is still written.
  *   ep_combine  y[t] = bf16( sum_j w[t][j] * e(t,j) ), fp32 fused multiply-add in
  *               pick order j from 0, rounded once to bf16 (nearest even), where
  *               e(t,j) = expert_out[dst_pos[t][j]] for a routed pick, ori_x[t]
@@ -94,7 +109,8 @@ typedef struct CUstream_st* ep_stream_t;
  *   local_expert_num * ep_world_size <= 2048), 1 <= k <= 16 (Constraints:
  *   0 < K <= 16), T = B / P <= M, Z, C, K >= 0 with Z + C + K <= 2048,
  *   E*P*M < 2^31 (int32 row ids), 16 <= d <= 32768 with d % 16 == 0,
- *   quant_mode in {0, 2}, smooth_rows in {0, 1}, layout in {0, 1}.  The T <= M
+ *   quant_mode in {0, 1, 2}, smooth_rows in {0, 1, E} (E > 1 needs quant_mode 1 or 2),
+ *   layout in {0, 1}.  The T <= M
  *   and E*P*M bounds apply to layout 0; layout 1 needs E*B < 2^31 and
  *   E*P <= 24576.
  */
@@ -108,8 +124,9 @@ typedef struct {
     int32_t n_zero;      /* zero experts  (ids E .. E+Z-1) */
     int32_t n_copy;      /* copy experts  (next C ids) */
     int32_t n_const;     /* constant experts (next K ids) */
-    int32_t quant_mode;  /* 0: bf16 pass-through; 2: dynamic per-token int8 */
-    int32_t smooth_rows; /* 0: no smooth scale; 1: one fp32 [d] vector may be given */
+    int32_t quant_mode;  /* 0: bf16 pass-through; 1: static int8; 2: dynamic per-token int8 */
+    int32_t smooth_rows; /* 0: no smooth scale; 1: one fp32 [d] vector may be given;
+                            E: one fp32 [d] row per routed expert ([E][d]) may be given */
     int32_t layout;      /* 0: low-latency [E][P*M][d] receive layout;
                             1: packed [B*k][d]: the rows of expert g start at
                                expert_offset[g], those of source rank r after the
@@ -130,9 +147,10 @@ typedef struct {
                              (the combine's source map); rows past a run's count
                              are not written.  rows = E*P*M (layout 0) or B*k
                              (layout 1; rows past expert_offset[E] unused) */
-    size_t recv_x;        /* [rows][d] int8 (quant_mode 2) or bf16 (quant_mode 0) */
-    size_t recv_scale;    /* fp32 [rows]        1/s of the row's token (quant_mode 2) */
-    size_t token_scale;   /* fp32 [B]           1/s per token (quant_mode 2) */
+    size_t recv_x;        /* [rows][d] int8 (quant_mode 1, 2) or bf16 (quant_mode 0) */
+    size_t recv_scale;    /* fp32 [rows]        1/s of the row's copy (quant_mode 2) */
+    size_t token_scale;   /* fp32 [B]           1/s per token (quant_mode 2; not
+                             written with a per-expert smooth scale) */
     size_t workspace;     /* scratch words; zero-filled by ep_buffer_create */
 } ep_buffer_sizes;
 
@@ -164,16 +182,23 @@ EP_API int ep_buffer_create(const ep_config* cfg, const ep_buffer_ptrs* ptrs, ep
 /* Free the host struct.  Device memory stays with the caller.  NULL is accepted. */
 EP_API int ep_buffer_destroy(ep_buffer* buf);
 
-/* Routing layout from topk_idx (int32 [B][k], device).  Writes expert_count,
- * expert_offset, recv_count, dst_pos and the written rows of recv_src. */
-EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, ep_stream_t stream);
+/* Routing layout from topk_idx (int32 [B][k], device) and the optional
+ * x_active_mask (uint8 [B], device, or NULL).  Writes expert_count, expert_offset,
+ * recv_count, dst_pos and the written rows of recv_src. */
+EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, const uint8_t* x_active_mask,
+                     ep_stream_t stream);
 
 /* Quantize (quant_mode 2) or pass through (0) x (bf16 [B][d], device) and scatter
  * every routed pick into recv_x (plus recv_scale, token_scale in mode 2), to the
  * receive rows of the latest ep_layout on this buffer.  smooth_scale is an fp32
- * [d] device vector or NULL; it must be NULL when cfg.smooth_rows == 0.
- * For T = B/P <= 256 the kernel derives those rows from the topk_idx passed to
- * that ep_layout (which must still hold the same ids) instead of reading dst_pos,
+ * device array of cfg.smooth_rows rows of d ([d], or [E][d] per routed expert) or
+ * NULL; it must be NULL when cfg.smooth_rows == 0.  With a per-expert scale the
+ * kernel works expert by expert over the receive rows of that ep_layout
+ * (recv_count, expert_offset and recv_src), so one must have run on this buffer
+ * (else EP_ERR_INVALID_ARG); it starts after the layout kernel has finished.  A
+ * receive row whose recv_src is not a token sets EP_ERRBIT_ROW_RANGE and is skipped.
+ * For T = B/P <= 256 the kernel derives those rows from the topk_idx (and mask)
+ * passed to that ep_layout (which must still hold the same values) instead of reading dst_pos,
  * so it can run alongside the layout kernel; it finishes only after the layout
  * kernel has.  Call it on the stream of that ep_layout, after it. */
 EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale,
@@ -185,23 +210,28 @@ EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_sc
  * others, which derives its receive rows from the routing itself), saving one
  * kernel launch on the critical path; otherwise the two kernels are launched in
  * order.  Arguments as for ep_layout and ep_dispatch. */
-EP_API int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx, const uint16_t* x,
+EP_API int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx,
+                              const uint8_t* x_active_mask, const uint16_t* x,
                               const float* smooth_scale, ep_stream_t stream);
 
 /* Weighted combine into y (bf16 [B][d], device).  expert_out: bf16 [E*P*M][d]
  * receive-layout expert outputs (may alias recv_x when quant_mode is 0);
  * topk_idx int32 [B][k] and topk_weights fp32 [B][k] as given to ep_layout;
+ * x_active_mask uint8 [B] or NULL, the mask given to ep_layout (inactive tokens
+ * get y = +0);
  * ori_x bf16 [B][d] (required when C + K > 0, else may be NULL);
  * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos.
  * y must not overlap any input. */
 EP_API int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,
-               const float* topk_weights, const uint16_t* ori_x, const uint16_t* a1,
-               const uint16_t* a2, const uint16_t* v, uint16_t* y, ep_stream_t stream);
+               const float* topk_weights, const uint8_t* x_active_mask, const uint16_t* ori_x,
+               const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
+               ep_stream_t stream);
 
 /* Layout for callers that cannot allocate device memory.  The pages have no
  * counterpart to this entry point; it exists for this library's users.
  *
- * Same outputs, bit for bit, as ep_layout on the same topk_idx, but without an
+ * Same outputs, bit for bit, as ep_layout on the same topk_idx with no
+ * x_active_mask (every token active), but without an
  * ep_buffer or a workspace: the caller passes only the inputs and the outputs
  * (device arrays sized as ep_buffer_size reports; cfg is validated the same
  * way).  Meant for callers that cannot allocate a workspace: an engine whose

@@ -57,6 +57,8 @@ def check_layout(rep, w, pipe, ref):
 
 def check_dispatch(rep, w, pipe, inp, ref_lay, sample_picks=None, rng=None):
     """quant_out / scales of the oracle vs the GPU receive rows of routed picks."""
+    if w.smooth == "expert" and inp["smooth"] is not None:
+        return check_dispatch_expert_smooth(rep, w, pipe, inp, ref_lay, sample_picks, rng)
     cfg = ocfg(w)
     q, ts = oracle.quantize(cfg, inp["x"], inp["smooth"])
     dp = ref_lay["dst_pos"]
@@ -69,7 +71,12 @@ def check_dispatch(rep, w, pipe, inp, ref_lay, sample_picks=None, rng=None):
     buf = pipe.buf
     rows_d = torch.from_numpy(rows.astype(np.int64)).to(buf.device)
     got = buf.recv_x[rows_d]
-    if w.quant_mode == 2:
+    if w.quant_mode == 1:
+        got = got.cpu().numpy()
+        bad = np.nonzero(np.any(got != q[tt], axis=1))[0]
+        rep.check(bad.size == 0, "%s: static int8 payload differs in %d of %d rows"
+                  % (w.name, bad.size, rows.size))
+    elif w.quant_mode == 2:
         got = got.cpu().numpy()
         bad = np.nonzero(np.any(got != q[tt], axis=1))[0]
         rep.check(bad.size == 0, "%s: int8 payload differs in %d of %d rows" % (w.name, bad.size, rows.size))
@@ -85,6 +92,34 @@ def check_dispatch(rep, w, pipe, inp, ref_lay, sample_picks=None, rng=None):
         rep.check(bad.size == 0, "%s: bf16 payload differs in %d of %d rows" % (w.name, bad.size, rows.size))
     rep.notes["dispatch_rows_checked"] = int(rows.size)
     return q, ts
+
+
+def check_dispatch_expert_smooth(rep, w, pipe, inp, ref_lay, sample_picks=None, rng=None):
+    """Per-expert smooth scale: every checked copy against the oracle's per-copy
+    quantization, computed on the checked tokens only into compact rows."""
+    dp = ref_lay["dst_pos"]
+    tt, jj = np.nonzero(dp >= 0)
+    if sample_picks is not None and tt.size > sample_picks:
+        sel = (rng or np.random.default_rng(0)).choice(tt.size, sample_picks, replace=False)
+        sel.sort()
+        tt, jj = tt[sel], jj[sel]
+    toks, tpos = np.unique(tt, return_inverse=True)
+    compact = np.full((toks.size, w.k), -1, np.int32)
+    compact[tpos, jj] = np.arange(tt.size, dtype=np.int32)
+    sub = ocfg(w, B=toks.size, P=1, M=max(toks.size, 1), layout=0)
+    rx, rsc = oracle.dispatch_expert_smooth(sub, inp["x"][toks], inp["smooth"],
+                                            inp["topk_idx"][toks], compact, max(tt.size, 1))
+    rows_d = torch.from_numpy(dp[tt, jj].astype(np.int64)).to(pipe.buf.device)
+    got = pipe.buf.recv_x[rows_d].cpu().numpy()
+    bad = np.nonzero(np.any(got != rx[:tt.size], axis=1))[0]
+    rep.check(bad.size == 0, "%s: per-expert int8 payload differs in %d of %d rows"
+              % (w.name, bad.size, tt.size))
+    if w.quant_mode == 2:
+        gs = pipe.buf.recv_scale[rows_d].cpu().numpy()
+        rep.check(np.array_equal(gs.view(np.uint32), rsc[:tt.size].view(np.uint32)),
+                  "%s: per-expert recv_scale differs" % w.name)
+    rep.notes["dispatch_rows_checked"] = int(tt.size)
+    return rx, rsc
 
 
 def place_expert_rows(w, pipe, ref_lay, tokens, seed_offset=0):
@@ -114,8 +149,9 @@ def check_combine(rep, w, pipe, inp, dev_inp, ref_lay, tokens=None, seed_offset=
     idx = inp["topk_idx"][tokens]
     wts = inp["topk_weights"][tokens]
     x = inp["x"][tokens]
+    act = None if inp.get("active") is None else inp["active"][tokens]
     y_ref = oracle.combine(sub, vals if vals.shape[0] else None, idx, wts, compact, x,
-                           inp["a1"], inp["a2"], inp["v"])
+                           inp["a1"], inp["a2"], inp["v"], active=act)
     compare_combine(rep, w.name, y_gpu, y_ref, idx, wts, compact, vals, x, w)
 
 

@@ -78,7 +78,7 @@ def test_sizes_bf16_specials():
     (dict(d=7160), abi.EP_ERR_INVALID_ARG),         # d % 16 != 0
     (dict(d=0), abi.EP_ERR_INVALID_ARG),
     (dict(d=65536), abi.EP_ERR_UNSUPPORTED),
-    (dict(quant_mode=1), abi.EP_ERR_INVALID_ARG),
+    (dict(quant_mode=-1), abi.EP_ERR_INVALID_ARG),
     (dict(quant_mode=3), abi.EP_ERR_INVALID_ARG),
     (dict(M=64), abi.EP_ERR_CAPACITY),              # T = 128 > M
     (dict(E=4096, P=8), abi.EP_ERR_UNSUPPORTED),     # E above 2048
@@ -88,12 +88,26 @@ def test_sizes_bf16_specials():
     (dict(layout=2), abi.EP_ERR_UNSUPPORTED),
     (dict(layout=1, E=2048, P=16, B=1024, M=64), abi.EP_ERR_UNSUPPORTED),   # E*P above the pack table
     (dict(smooth_rows=2), abi.EP_ERR_INVALID_ARG),
+    (dict(smooth_rows=64, quant_mode=0), abi.EP_ERR_INVALID_ARG),  # per-expert scale needs int8
     (dict(P=0), abi.EP_ERR_INVALID_ARG),
 ])
 def test_bad_configs(kw, status):
     with pytest.raises(abi.EPError) as ei:
         abi.ep_buffer_size(cfg(**kw))
     assert ei.value.status == status
+
+
+def test_sizes_static_int8():
+    """quant_mode 1 (static int8): an int8 payload and no scales."""
+    s = abi.ep_buffer_size(cfg(quant_mode=1))
+    rows = 256 * 8 * 128
+    assert s.recv_x == rows * 7168
+    assert s.recv_scale == 0 and s.token_scale == 0
+
+
+def test_sizes_expert_smooth():
+    """A per-expert smooth scale (smooth_rows = E) changes no buffer size."""
+    assert abi.ep_buffer_size(cfg(smooth_rows=256)).recv_x == abi.ep_buffer_size(cfg()).recv_x
 
 
 def test_sizes_packed():

@@ -62,7 +62,7 @@ def full_check(w, dev, inp=None, tokens=None, sample_picks=None, separate=True, 
         pipe.layout(dev_inp)
         pipe.dispatch(dev_inp)
     err = pipe.buf.check()
-    ref = oracle.layout(gp.ocfg(w), inp["topk_idx"])
+    ref = oracle.layout(gp.ocfg(w), inp["topk_idx"], active=inp.get("active"))
     rep.check(err == ref["err"], "%s: device error bits %#x, oracle %#x" % (w.name, err, ref["err"]))
     gp.check_layout(rep, w, pipe, ref)
     gp.check_dispatch(rep, w, pipe, inp, ref, sample_picks=sample_picks)
@@ -206,6 +206,192 @@ def test_packed_dirty(dev):
     gp.check_dispatch(rep, w, pipe, inp, ref)
     gp.check_combine(rep, w, pipe, inp, dev_inp, ref)
     rep.assert_ok()
+
+
+# ----------------------------------------------------------------------------- per-expert smooth scale
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_expert", dict(base="tiny_q2")),                       # T = 128: rows from the routing
+    ("decode_expert_smooth", dict()),                            # decode shape, T = 128
+    ("skewed_expert", dict(base="skewed")),                      # T = 1024: rows from dst_pos, specials
+    ("decode_expert_packed", dict(base="decode", layout=1)),     # packed rows
+])
+def test_expert_smooth(dev, name, kw):
+    """Per-expert smooth scale [E, d]: every routed copy quantized on its own."""
+    kw = dict(kw)
+    base = kw.pop("base", None)
+    w = wl.get(name) if base is None else wl.get(base).with_(name=name, smooth="expert", **kw)
+    full_check(w, dev)
+    full_check(w.with_(name=name + "_fused"), dev, fused=True)
+
+
+@pytest.mark.parametrize("d", [16, 272, 32768])
+def test_expert_smooth_widths(dev, d):
+    w = wl.Workload("expert_d%d" % d, B=3 * 37, d=d, k=3, P=3, M=40, E=9, quant_mode=2,
+                    smooth="expert", seed=d)
+    full_check(w, dev)
+
+
+def test_expert_smooth_dirty(dev):
+    """Bad and repeated ids with a per-expert scale: those picks get no row, the
+    others are quantized per copy."""
+    w = wl.Workload("ragged_expert", B=111, d=272, k=3, P=3, M=40, E=9, n_zero=1, n_copy=1,
+                    n_const=1, quant_mode=2, smooth="expert", seed=9)
+    inp = wl.generate(w)
+    rng = np.random.default_rng(9)
+    idx = np.stack([rng.permutation(w.E_tot)[:w.k] for _ in range(w.B)]).astype(np.int32)
+    idx[2, 0] = -1
+    idx[5, 1] = w.E_tot
+    idx[11] = [3, 7, 3]
+    inp["topk_idx"] = idx
+    inp["x"][20] = 0                   # degenerate copies: q = 0, scale 0
+    for name, fused in (("dirty", False), ("dirty_fused", True)):
+        dev_inp = runner.to_device(inp, dev)
+        pipe = runner.Pipeline(w, dev, alias_expert_out=False)
+        if fused:
+            pipe.layout_dispatch(dev_inp)
+        else:
+            pipe.layout(dev_inp)
+            pipe.dispatch(dev_inp)
+        err = pipe.buf.check()
+        ref = oracle.layout(gp.ocfg(w), idx)
+        assert err == ref["err"] == (oracle.ERR_BAD_ID | oracle.ERR_DUP_ID), name
+        rep = gp.Report()
+        gp.check_layout(rep, w, pipe, ref)
+        gp.check_dispatch(rep, w, pipe, inp, ref)
+        gp.check_combine(rep, w, pipe, inp, dev_inp, ref)
+        rep.assert_ok()
+
+
+def test_expert_smooth_identical_rows_match_token_scale(dev):
+    """Closed form on the GPU: an [E, d] scale whose rows are all one [d] vector
+    gives the same receive rows and scales as that vector given per token."""
+    w = wl.get("decode").with_(name="decode_same_rows", smooth="rand")
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev)
+    we = w.with_(smooth="expert")
+    pipe_e = runner.Pipeline(we, dev)
+    dev_e = dict(dev_inp)
+    dev_e["smooth"] = dev_inp["smooth"].expand(w.E, w.d).contiguous()
+    pipe.layout(dev_inp)
+    pipe.dispatch(dev_inp)
+    pipe_e.layout(dev_e)
+    pipe_e.dispatch(dev_e)
+    torch.cuda.synchronize()
+    dp = pipe.buf.dst_pos.flatten()
+    rows = dp[dp >= 0].long()
+    assert torch.equal(pipe.buf.recv_x[rows], pipe_e.buf.recv_x[rows])
+    assert torch.equal(pipe.buf.recv_scale[rows], pipe_e.buf.recv_scale[rows])
+    assert pipe.buf.check() == 0 and pipe_e.buf.check() == 0
+
+
+def test_expert_smooth_needs_layout(dev):
+    """A per-expert scale names the copies' experts through the latest layout's
+    routing: ep_dispatch before any ep_layout is refused on the host."""
+    from combine_ep_layout_12_b200 import _binding as abi
+    w = small("expert_no_layout", smooth="expert")
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    buf = EPBuffer(w, device=dev)
+    with pytest.raises(abi.EPError) as ei:
+        buf.dispatch(dev_inp["x"], dev_inp["smooth"])
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- static int8 and x_active_mask
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_static", dict(base="tiny_q2", quant_mode=1, smooth="rand")),
+    ("tiny_static_noscale", dict(base="tiny_q2", quant_mode=1, smooth="none")),
+    ("decode_static", dict()),
+    ("skewed_static", dict(base="skewed", quant_mode=1, smooth="rand")),
+    ("decode_static_packed", dict(base="decode", quant_mode=1, smooth="rand", layout=1)),
+    ("decode_static_expert", dict(base="decode", quant_mode=1, smooth="expert")),
+])
+def test_static_quant(dev, name, kw):
+    """quant_mode 1: CastToInt8(CastToFp32(x) * scales), no scale sent."""
+    kw = dict(kw)
+    base = kw.pop("base", None)
+    w = wl.get(name) if base is None else wl.get(base).with_(name=name, **kw)
+    full_check(w, dev)
+    full_check(w.with_(name=name + "_fused"), dev, fused=True)
+
+
+def test_static_quant_closed_forms(dev):
+    """Integers pass through, x.5 ties go to even, beyond [-128, 127] saturates."""
+    w = wl.Workload("static_cf", B=4, d=32, k=2, P=2, M=2, E=4, quant_mode=1, seed=3)
+    inp = wl.generate(w)
+    vals = np.array([0, 1, -1, 2.5, 3.5, -2.5, -0.5, 0.5, 126, 127, 127.5, 128, 300,
+                     -128, -128.5, -129, -300, 1.5, -1.5, 64.25], np.float32)
+    want = np.array([0, 1, -1, 2, 4, -2, 0, 0, 126, 127, 127, 127, 127, -128, -128, -128, -128,
+                     2, -2, 64], np.int8)
+    xv = np.zeros((w.B, w.d), np.float32)
+    xv[:, :vals.size] = vals
+    inp["x"] = wl.f32_to_bf16_bits(xv)
+    pipe, *_ = full_check(w, dev, inp=inp)
+    dp = pipe.buf.dst_pos.flatten()
+    rows = dp[dp >= 0].long()
+    got = pipe.buf.recv_x[rows][:, :vals.size].cpu().numpy()
+    assert (got == want[None, :]).all()
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_active", dict(base="tiny_q2", active_frac=0.5)),
+    ("decode_active", dict()),                                          # T = 128, one grid
+    ("decode_active_bf16", dict(base="decode", quant_mode=0, active_frac=0.75)),
+    ("skewed_active", dict(base="skewed", active_frac=0.6)),            # multi-CTA layout, specials
+    ("decode_active_packed", dict(base="decode", active_frac=0.75, layout=1)),
+    ("sweep_T256_active", dict(base="sweep_T256_q2", active_frac=0.8)),
+    ("decode_active_expert", dict(base="decode", active_frac=0.75, smooth="expert")),
+    ("decode_active_none", dict(base="decode", active_frac=0.0)),
+])
+def test_active_mask(dev, name, kw):
+    """x_active_mask: inactive tokens route nothing, count nowhere and get y = +0."""
+    kw = dict(kw)
+    base = kw.pop("base", None)
+    w = wl.get(name) if base is None else wl.get(base).with_(name=name, **kw)
+    pipe, dev_inp, inp, ref = full_check(w, dev)
+    off = np.nonzero(inp["active"] == 0)[0]
+    if off.size:
+        y = pipe.y[torch.from_numpy(off).to(dev)]
+        assert int(y.view(torch.int16).abs().max()) == 0
+    full_check(w.with_(name=name + "_fused"), dev, fused=True)
+
+
+def test_active_mask_ignores_bad_ids_of_inactive_tokens(dev):
+    """An inactive token's ids are not looked at: bad or repeated ids there raise
+    no error bit, while the same ids in an active token do."""
+    w = wl.Workload("active_dirty", B=111, d=272, k=3, P=3, M=40, E=9, n_zero=1, n_copy=1,
+                    n_const=1, quant_mode=2, smooth="rand", seed=13, active_frac=1.0)
+    inp = wl.generate(w)
+    rng = np.random.default_rng(13)
+    idx = np.stack([rng.permutation(w.E_tot)[:w.k] for _ in range(w.B)]).astype(np.int32)
+    idx[5, 1] = w.E_tot + 4
+    idx[11] = [3, 7, 3]
+    inp["topk_idx"] = idx
+    for act5, want in ((0, oracle.ERR_DUP_ID), (1, oracle.ERR_DUP_ID | oracle.ERR_BAD_ID)):
+        inp["active"] = np.ones(w.B, np.uint8)
+        inp["active"][5] = act5
+        inp["active"][40:50] = 0
+        for fused in (False, True):
+            dev_inp = runner.to_device(inp, dev)
+            pipe = runner.Pipeline(w, dev, alias_expert_out=False)
+            if fused:
+                pipe.layout_dispatch(dev_inp)
+            else:
+                pipe.layout(dev_inp)
+                pipe.dispatch(dev_inp)
+            err = pipe.buf.check()
+            ref = oracle.layout(gp.ocfg(w), idx, active=inp["active"])
+            assert err == ref["err"] == want
+            rep = gp.Report()
+            gp.check_layout(rep, w, pipe, ref)
+            gp.check_dispatch(rep, w, pipe, inp, ref)
+            gp.check_combine(rep, w, pipe, inp, dev_inp, ref)
+            rep.assert_ok()
 
 
 # ----------------------------------------------------------------------------- fused call
