@@ -41,10 +41,11 @@ METRIC = "dispatch+combine HBM GB/s and tokens/s at d=7168,E=256,k=8; % of B200 
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 PROFILES = os.path.join(ROOT, "profiles")
-KERNEL_SOURCES = {
-    "layout": "combine_ep_layout_12_b200/csrc/ep_layout.cu",
-    "dispatch": "combine_ep_layout_12_b200/csrc/ep_dispatch.cu",
-    "combine": "combine_ep_layout_12_b200/csrc/ep_combine.cu",
+_CSRC = "combine_ep_layout_12_b200/csrc/"
+KERNEL_SOURCES = {  # every source file a kernel's code comes from
+    "layout": [_CSRC + f for f in ("ep_layout.cu", "ep_layout_dev.cuh", "ep_internal.cuh")],
+    "dispatch": [_CSRC + f for f in ("ep_dispatch.cu", "ep_dispatch_dev.cuh", "ep_internal.cuh")],
+    "combine": [_CSRC + f for f in ("ep_combine.cu", "ep_internal.cuh")],
 }
 
 
@@ -197,8 +198,11 @@ def measured_peak():
 
 
 def source_hash(name):
-    with open(os.path.join(ROOT, KERNEL_SOURCES[name]), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[name]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload, kernel):

@@ -16,6 +16,8 @@
 // warp shuffles and one shared-memory pass, quantized in registers, and written
 // to each of the token's k receive rows with 16-byte stores.  The read happens
 // once per token; the k writes are the bulk of the traffic.
+#include <mutex>
+
 #include "ep_internal.cuh"
 #include "ep_dispatch_dev.cuh"
 
@@ -62,13 +64,16 @@ cudaError_t launch_int8(int U, dim3 grid, dim3 block, cudaStream_t stream, const
 // makes the kernel bound by L2 reads of the table.  Instead a CTA takes one
 // expert g and a share of its receive rows: it stages smooth[g] in shared memory
 // once, finds the source token of each of its rows through recv_src, and
-// quantizes the rows one at a time with all its threads.  A thread holds GP
-// groups of 4 elements of the row in registers (the x row is read once, from L2),
-// the absmax is one CTA reduction behind one barrier (two alternating sets of
-// reduction slots), and the next row's x is loaded before that barrier so its
-// latency overlaps the reduction.  Loads, stores and the float4 shared-memory
-// reads are all lane-contiguous.  The receive rows come from the layout
-// (recv_count, recv_src, expert_offset), so the kernel waits for it first.
+// quantizes the rows one at a time with all its threads.  Per-copy quantization
+// does k times the arithmetic of the per-token form, so the loop is written for
+// few instructions per element: a thread owns GP units of 8 elements (one 16-byte
+// x load and one 8-byte store per unit), x_fp32 is formed once per element and
+// kept in registers for the cast, the smooth row sits in two float4 planes so
+// the shared-memory reads are conflict-free, and the absmax is one CTA reduction
+// behind one barrier (two alternating slot sets).  The next row's x is loaded
+// before that barrier so its latency overlaps the reduction.  The receive rows
+// come from the layout (recv_count, recv_src, expert_offset), so the kernel
+// waits for it first.
 // ---------------------------------------------------------------------------
 struct ExpertArgs {
     const uint16_t* x;             // [B][d]
@@ -83,32 +88,38 @@ struct ExpertArgs {
     int B, d, P, M, E, parts, layout;
 };
 
-template <int GP>
-__device__ __forceinline__ void load_x_groups(const ExpertArgs& a, int t, int nq, uint2 (&v)[GP]) {
-    const uint2* xr = reinterpret_cast<const uint2*>(a.x + (size_t)(t < 0 ? 0 : t) * a.d);
+// EXACT: the CTA's threads times GP cover the d / 8 units exactly (no bounds checks).
+template <int GP, bool EXACT>
+__device__ __forceinline__ void load_x_units(const ExpertArgs& a, int t, int nu, uint4 (&v)[GP]) {
+    const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(t < 0 ? 0 : t) * a.d);
 #pragma unroll
     for (int m = 0; m < GP; ++m) {
-        const int q = threadIdx.x + m * blockDim.x;
-        v[m] = (t >= 0 && q < nq) ? __ldg(xr + q) : make_uint2(0, 0);
+        const int u = threadIdx.x + m * blockDim.x;
+        v[m] = (t >= 0 && (EXACT || u < nu)) ? __ldg(xr + u) : make_uint4(0, 0, 0, 0);
     }
 }
 
-template <int GP, int MAXT, bool STATIC>
+template <int GP, int MAXT, bool STATIC, bool EXACT>
 __global__ void __launch_bounds__(MAXT) dispatch_expert_major_kernel(ExpertArgs a) {
-    extern __shared__ float4 s_sm4[];                                          // [d / 4]
+    extern __shared__ float4 s_sm4[];                                        // 2 planes of [d / 8]
     const int NT = blockDim.x;
-    long long* s_row = reinterpret_cast<long long*>(s_sm4 + (a.d >> 2));    // [NT]
+    const int nu = a.d >> 3;
+    float4* s_lo = s_sm4;                                                    // elements 8u .. 8u+3
+    float4* s_hi = s_sm4 + nu;                                               // elements 8u+4 .. 8u+7
+    long long* s_row = reinterpret_cast<long long*>(s_sm4 + 2 * nu);        // [NT]
     int* s_t = reinterpret_cast<int*>(s_row + NT);                           // [NT]
     int* s_pre = s_t + NT;                                                   // [P + 1]
     __shared__ float s_red[2][32];
     pdl_wait();
     pdl_launch_dependents();
     const int g = blockIdx.x / a.parts, part = blockIdx.x - g * a.parts;
-    const int nq = a.d >> 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = NT >> 5;
 
     const float4* srow = reinterpret_cast<const float4*>(a.smooth + (size_t)g * a.d);
-    for (int q = threadIdx.x; q < nq; q += NT) s_sm4[q] = __ldg(srow + q);
+    for (int u = threadIdx.x; u < nu; u += NT) {
+        s_lo[u] = __ldg(srow + 2 * u);
+        s_hi[u] = __ldg(srow + 2 * u + 1);
+    }
     if (a.layout == 0 && warp == 0) {
         // exclusive prefix over source ranks of this expert's row counts
         int run = 0;
@@ -157,26 +168,38 @@ __global__ void __launch_bounds__(MAXT) dispatch_expert_major_kernel(ExpertArgs 
             s_t[threadIdx.x] = ok ? t : -1;
         }
         __syncthreads();
-        uint2 cur[GP], nxt[GP];
-        load_x_groups<GP>(a, s_t[0], nq, cur);
+        uint4 cur[GP], nxt[GP];
+        load_x_units<GP, EXACT>(a, s_t[0], nu, cur);
         for (int j = 0; j < nb; ++j) {
             const int t = s_t[j];
             const long long row = s_row[j];
-            if (j + 1 < nb) load_x_groups<GP>(a, s_t[j + 1], nq, nxt);
+            // x_fp32 = fp32(x) * smooth[g], formed once per element and kept for the cast
+            float f[GP][8];
+            float amax = 0.0f;
+#pragma unroll
+            for (int m = 0; m < GP; ++m) {
+                const int u = threadIdx.x + m * NT;
+                const bool in = EXACT || u < nu;
+                const float4 lo4 = in ? s_lo[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float4 hi4 = in ? s_hi[u] : make_float4(0.f, 0.f, 0.f, 0.f);
+                f[m][0] = __fmul_rn(bf16lo(cur[m].x), lo4.x);
+                f[m][1] = __fmul_rn(bf16hi(cur[m].x), lo4.y);
+                f[m][2] = __fmul_rn(bf16lo(cur[m].y), lo4.z);
+                f[m][3] = __fmul_rn(bf16hi(cur[m].y), lo4.w);
+                f[m][4] = __fmul_rn(bf16lo(cur[m].z), hi4.x);
+                f[m][5] = __fmul_rn(bf16hi(cur[m].z), hi4.y);
+                f[m][6] = __fmul_rn(bf16lo(cur[m].w), hi4.z);
+                f[m][7] = __fmul_rn(bf16hi(cur[m].w), hi4.w);
+                if (!STATIC) {
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2)
+                        amax = fmaxf(amax, fmaxf(fabsf(f[m][e]), fabsf(f[m][e + 1])));
+                }
+            }
+            if (j + 1 < nb) load_x_units<GP, EXACT>(a, s_t[j + 1], nu, nxt);
             float s = 1.0f;
             bool degenerate = false;
             if (!STATIC) {
-                float amax = 0.0f;
-#pragma unroll
-                for (int m = 0; m < GP; ++m) {
-                    const int q = threadIdx.x + m * NT;
-                    if (q >= nq) continue;
-                    const float4 sm = s_sm4[q];
-                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(__fmul_rn(bf16lo(cur[m].x), sm.x)),
-                                                   fabsf(__fmul_rn(bf16hi(cur[m].x), sm.y))),
-                                             fmaxf(fabsf(__fmul_rn(bf16lo(cur[m].y), sm.z)),
-                                                   fabsf(__fmul_rn(bf16hi(cur[m].y), sm.w)))));
-                }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
                 if (lane == 0) s_red[par][warp] = amax;
@@ -188,19 +211,23 @@ __global__ void __launch_bounds__(MAXT) dispatch_expert_major_kernel(ExpertArgs 
                 degenerate = (amax == 0.0f) || isinf(s);
             }
             if (t >= 0) {
-                uint32_t* out = reinterpret_cast<uint32_t*>(a.recv_x + row * a.d);
+                uint2* out = reinterpret_cast<uint2*>(a.recv_x + row * a.d);
 #pragma unroll
                 for (int m = 0; m < GP; ++m) {
-                    const int q = threadIdx.x + m * NT;
-                    if (q >= nq) continue;
-                    const float4 sm = s_sm4[q];
-                    float f0 = __fmul_rn(bf16lo(cur[m].x), sm.x), f1 = __fmul_rn(bf16hi(cur[m].x), sm.y);
-                    float f2 = __fmul_rn(bf16lo(cur[m].y), sm.z), f3 = __fmul_rn(bf16hi(cur[m].y), sm.w);
-                    if (!STATIC) {
-                        f0 = __fmul_rn(f0, s); f1 = __fmul_rn(f1, s);
-                        f2 = __fmul_rn(f2, s); f3 = __fmul_rn(f3, s);
+                    const int u = threadIdx.x + m * NT;
+                    if (!EXACT && u >= nu) continue;
+                    uint2 word;
+                    if (STATIC) {
+                        word.x = cvt_s8x4(f[m][0], f[m][1], f[m][2], f[m][3]);
+                        word.y = cvt_s8x4(f[m][4], f[m][5], f[m][6], f[m][7]);
+                    } else {
+                        word.x = cvt_s8x4_unclamped(__fmul_rn(f[m][0], s), __fmul_rn(f[m][1], s),
+                                                    __fmul_rn(f[m][2], s), __fmul_rn(f[m][3], s));
+                        word.y = cvt_s8x4_unclamped(__fmul_rn(f[m][4], s), __fmul_rn(f[m][5], s),
+                                                    __fmul_rn(f[m][6], s), __fmul_rn(f[m][7], s));
+                        if (degenerate) word = make_uint2(0, 0);
                     }
-                    out[q] = degenerate ? 0u : cvt_s8x4(f0, f1, f2, f3);
+                    out[u] = word;
                 }
                 if (!STATIC && threadIdx.x == 0)
                     a.recv_scale[row] = degenerate ? 0.0f : __fdiv_rn(1.0f, s);
@@ -212,29 +239,40 @@ __global__ void __launch_bounds__(MAXT) dispatch_expert_major_kernel(ExpertArgs 
     }
 }
 
-// GP groups per thread; up to 256 threads, or 1024 for rows above 8192 elements.
-template <bool STATIC>
-cudaError_t launch_expert_gp(int GP, int NT, dim3 grid, size_t smem, cudaStream_t stream,
-                             const ExpertArgs& a) {
-    const dim3 block((unsigned)NT);
+using ExpertKernel = void (*)(ExpertArgs);
+
+// GP units of 8 elements per thread, up to 256 threads (1024 for rows above 8192
+// elements), and whether NT * GP covers the row exactly.
+ExpertKernel pick_expert_kernel(bool st, int GP, int NT, bool exact) {
+#define EP_EXPERT_K(G, T)                                                                          \
+    (st ? (exact ? dispatch_expert_major_kernel<G, T, true, true> : dispatch_expert_major_kernel<G, T, true, false>) \
+        : (exact ? dispatch_expert_major_kernel<G, T, false, true> : dispatch_expert_major_kernel<G, T, false, false>))
     switch (GP) {
-        case 1: return launch_pdl(dispatch_expert_major_kernel<1, 256, STATIC>, grid, block, smem, stream, a);
-        case 2: return launch_pdl(dispatch_expert_major_kernel<2, 256, STATIC>, grid, block, smem, stream, a);
-        case 4: return launch_pdl(dispatch_expert_major_kernel<4, 256, STATIC>, grid, block, smem, stream, a);
-        default:
-            return NT <= 256
-                ? launch_pdl(dispatch_expert_major_kernel<8, 256, STATIC>, grid, block, smem, stream, a)
-                : launch_pdl(dispatch_expert_major_kernel<8, 1024, STATIC>, grid, block, smem, stream, a);
+        case 1: return EP_EXPERT_K(1, 256);
+        case 2: return EP_EXPERT_K(2, 256);
+        default: return NT <= 256 ? EP_EXPERT_K(4, 256) : EP_EXPERT_K(4, 1024);
     }
+#undef EP_EXPERT_K
 }
 
-template <int GP, int MAXT>
-cudaError_t set_expert_smem(int cap) {
-    cudaError_t e = cudaFuncSetAttribute(dispatch_expert_major_kernel<GP, MAXT, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(dispatch_expert_major_kernel<GP, MAXT, true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, cap);
+// Resident CTAs per SM of one kernel configuration, queried once per device and
+// configuration (the result depends only on the kernel's resources).
+int expert_occupancy(ExpertKernel kern, int NT, size_t smem) {
+    struct Entry { int dev; ExpertKernel k; int nt; size_t smem; int occ; };
+    static Entry cache[32];
+    static int n_cache = 0;
+    static std::mutex mu;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n_cache; ++i)
+        if (cache[i].dev == dev && cache[i].k == kern && cache[i].nt == NT && cache[i].smem == smem)
+            return cache[i].occ;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, NT, smem) != cudaSuccess || occ < 1)
+        occ = 1;
+    if (n_cache < 32) cache[n_cache++] = {dev, kern, NT, smem, occ};
+    return occ;
 }
 
 int launch_dispatch_expert(const Shape& sh, const ep_buffer_ptrs& p, const uint16_t* x,
@@ -250,36 +288,29 @@ int launch_dispatch_expert(const Shape& sh, const ep_buffer_ptrs& p, const uint1
     a.err = &reinterpret_cast<WsHeader*>(p.workspace)->err;
     a.rows = sh.rows;
     a.B = sh.B; a.d = sh.d; a.P = sh.P; a.M = sh.M; a.E = sh.E; a.layout = sh.layout;
-    // groups of 4 elements per thread: the smallest GP in {1, 2, 4, 8} with at most
-    // 256 threads, else GP = 8 with up to 1024 threads (d <= 32768)
-    const int nq = sh.d / 4;
+    // units of 8 elements per thread: the smallest GP in {1, 2, 4} with at most 256
+    // threads, else GP = 4 with up to 1024 threads (d <= 32768)
+    const int nu = sh.d / 8;
     int GP = 1;
-    while (GP < 8 && (nq + GP - 1) / GP > 256) GP *= 2;
-    int NT = (nq + GP - 1) / GP;
+    while (GP < 4 && (nu + GP - 1) / GP > 256) GP *= 2;
+    int NT = (nu + GP - 1) / GP;
     NT = ((NT + 31) / 32) * 32;
     if (NT > 1024) return EP_ERR_UNSUPPORTED;
-    // about four CTAs per SM in total, split evenly over the experts
-    const long long target = (long long)num_sms() * 4;
+    const bool exact = NT * GP == nu;
+    const ExpertKernel kern = pick_expert_kernel(sh.quant_mode == 1, GP, NT, exact);
+    const size_t smem = sizeof(float) * (size_t)sh.d + (sizeof(long long) + sizeof(int)) * (size_t)NT +
+                        sizeof(int) * ((size_t)sh.P + 1);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return EP_ERR_CUDA;
+    // about four waves of resident CTAs, split evenly over the experts
+    const int occ = expert_occupancy(kern, NT, smem);
+    const long long target = 4LL * num_sms() * occ;
     long long parts = (target + sh.E - 1) / sh.E;
     if (parts < 1) parts = 1;
     a.parts = (int)parts;
-    const size_t smem = sizeof(float) * (size_t)sh.d + (sizeof(long long) + sizeof(int)) * (size_t)NT +
-                        sizeof(int) * ((size_t)sh.P + 1);
-    static bool attr_set[64] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-        const int cap = (int)(sizeof(float) * kMaxD + (sizeof(long long) + sizeof(int)) * 1024 +
-                              sizeof(int) * (kMaxE + 1));
-        if (set_expert_smem<1, 256>(cap) || set_expert_smem<2, 256>(cap) ||
-            set_expert_smem<4, 256>(cap) || set_expert_smem<8, 256>(cap) ||
-            set_expert_smem<8, 1024>(cap))
-            return EP_ERR_CUDA;
-        attr_set[dev] = true;
-    }
     const dim3 grid((unsigned)((long long)sh.E * a.parts));
-    const cudaError_t e = sh.quant_mode == 1 ? launch_expert_gp<true>(GP, NT, grid, smem, stream, a)
-                                             : launch_expert_gp<false>(GP, NT, grid, smem, stream, a);
+    const cudaError_t e = launch_pdl(kern, grid, dim3((unsigned)NT), smem, stream, a);
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 

@@ -84,6 +84,19 @@ __device__ __forceinline__ uint32_t cvt_s8x4(float a, float b, float c, float d)
     return __byte_perm(lo, hi, 0x5410);
 }
 
+// The same for values already known to lie within [-127.5, 127.5): in dynamic
+// quantization |x_fp32 * s| <= amax * fl(127 / amax), which is at most
+// 127 * (1 + 2^-24)^2 after the two roundings, so the saturation never acts and
+// the clamp is left out.
+__device__ __forceinline__ uint32_t s8_byte_word_unclamped(float v) {
+    return __float_as_uint(__fadd_rn(v, 12582912.0f));
+}
+__device__ __forceinline__ uint32_t cvt_s8x4_unclamped(float a, float b, float c, float d) {
+    const uint32_t lo = __byte_perm(s8_byte_word_unclamped(a), s8_byte_word_unclamped(b), 0x0040);
+    const uint32_t hi = __byte_perm(s8_byte_word_unclamped(c), s8_byte_word_unclamped(d), 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
+}
+
 // quant_mode 2 (dynamic) or 1 (STATIC: q = CastToInt8(x_fp32), no absmax and no
 // scale): a unit is 16 elements (two 16-byte bf16 loads -> one 16-byte int8 store).
 template <int U, bool STATIC>
@@ -157,8 +170,15 @@ __device__ __forceinline__ void dispatch_int8_body(const DispatchArgs& a, int t)
 #pragma unroll
             for (int e = 0; e < 16; ++e) f[e] = __fmul_rn(f[e], s);
         }
-        uint4 v = make_uint4(cvt_s8x4(f[0], f[1], f[2], f[3]), cvt_s8x4(f[4], f[5], f[6], f[7]),
-                             cvt_s8x4(f[8], f[9], f[10], f[11]), cvt_s8x4(f[12], f[13], f[14], f[15]));
+        uint4 v;
+        if (STATIC)
+            v = make_uint4(cvt_s8x4(f[0], f[1], f[2], f[3]), cvt_s8x4(f[4], f[5], f[6], f[7]),
+                           cvt_s8x4(f[8], f[9], f[10], f[11]), cvt_s8x4(f[12], f[13], f[14], f[15]));
+        else
+            v = make_uint4(cvt_s8x4_unclamped(f[0], f[1], f[2], f[3]),
+                           cvt_s8x4_unclamped(f[4], f[5], f[6], f[7]),
+                           cvt_s8x4_unclamped(f[8], f[9], f[10], f[11]),
+                           cvt_s8x4_unclamped(f[12], f[13], f[14], f[15]));
         if (degenerate) v = make_uint4(0, 0, 0, 0);
         for (int j = 0; j < a.k; ++j) {
             const int row = s_rows[j];

@@ -226,9 +226,11 @@ def test_expert_smooth(dev, name, kw):
     full_check(w.with_(name=name + "_fused"), dev, fused=True)
 
 
+@pytest.mark.parametrize("qm", [1, 2])
 @pytest.mark.parametrize("d", [16, 272, 32768])
-def test_expert_smooth_widths(dev, d):
-    w = wl.Workload("expert_d%d" % d, B=3 * 37, d=d, k=3, P=3, M=40, E=9, quant_mode=2,
+def test_expert_smooth_widths(dev, d, qm):
+    """Rows that do not tile the CTA (d = 16, 272) and the widest rows (1024 threads)."""
+    w = wl.Workload("expert_d%d_q%d" % (d, qm), B=3 * 37, d=d, k=3, P=3, M=40, E=9, quant_mode=qm,
                     smooth="expert", seed=d)
     full_check(w, dev)
 
