@@ -52,10 +52,11 @@ class EPBuffer:
     Views: expert_count [E_tot], expert_offset [E_tot+1], recv_count [E, P],
     dst_pos [B, k], recv_src [rows], recv_x [rows, d] (int8 or bf16),
     recv_scale [rows], token_scale [B]; rows = E*P*M (low-latency layout) or
-    B*k (packed layout).
+    B*k (packed layout).  alloc(shape, dtype) -> tensor, if given, provides the
+    arrays (e.g. carved out of larger allocations); default torch.empty.
     """
 
-    def __init__(self, cfg, device=None):
+    def __init__(self, cfg, device=None, alloc=None):
         if not isinstance(cfg, abi.ep_config):
             cfg = make_config(cfg.B, cfg.d, cfg.k, cfg.P, cfg.M, cfg.E, cfg.n_zero, cfg.n_copy,
                               cfg.n_const, cfg.quant_mode, getattr(cfg, "smooth_rows", 1),
@@ -71,17 +72,20 @@ class EPBuffer:
         self.E_tot = c.E + c.n_zero + c.n_copy + c.n_const
         self.rows = c.B * c.k if c.layout == 1 else c.E * c.P * c.M
         dev = self.device
-        self.expert_count = torch.empty(self.E_tot, dtype=torch.int32, device=dev)
-        self.expert_offset = torch.empty(self.E_tot + 1, dtype=torch.int32, device=dev)
-        self.recv_count = torch.empty((c.E, c.P), dtype=torch.int32, device=dev)
-        self.dst_pos = torch.empty((c.B, c.k), dtype=torch.int32, device=dev)
-        self.recv_src = torch.empty(self.rows, dtype=torch.int32, device=dev)
+        if alloc is None:
+            def alloc(shape, dtype):
+                return torch.empty(shape, dtype=dtype, device=dev)
+        self.expert_count = alloc((self.E_tot,), torch.int32)
+        self.expert_offset = alloc((self.E_tot + 1,), torch.int32)
+        self.recv_count = alloc((c.E, c.P), torch.int32)
+        self.dst_pos = alloc((c.B, c.k), torch.int32)
+        self.recv_src = alloc((self.rows,), torch.int32)
         xdt = torch.int8 if c.quant_mode != 0 else torch.bfloat16
-        self.recv_x = torch.empty((self.rows, c.d), dtype=xdt, device=dev)
+        self.recv_x = alloc((self.rows, c.d), xdt)
         q = c.quant_mode == 2
-        self.recv_scale = torch.empty(self.rows, dtype=torch.float32, device=dev) if q else None
-        self.token_scale = torch.empty(c.B, dtype=torch.float32, device=dev) if q else None
-        self.workspace = torch.empty(self.sizes["workspace"], dtype=torch.uint8, device=dev)
+        self.recv_scale = alloc((self.rows,), torch.float32) if q else None
+        self.token_scale = alloc((c.B,), torch.float32) if q else None
+        self.workspace = alloc((self.sizes["workspace"],), torch.uint8)
         ptrs = abi.ep_buffer_ptrs(*[_ptr(getattr(self, n)) for n in abi.BUFFER_FIELDS])
         with torch.cuda.device(dev):
             self.handle = ep_buffer_create(cfg, ptrs)

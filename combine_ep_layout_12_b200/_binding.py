@@ -43,19 +43,37 @@ class EPError(RuntimeError):
         super().__init__("%s failed: %s (status %d)" % (where, ep_status_str(status), status))
 
 
-_lib = None
+LIB_CHECKED_PATH = os.path.join(_PKG, "libep_checked.so")
+ERRBIT_CHECKED = 0x8
+
+_libs = {}
+_use_checked = False
+
+
+def use_checked(flag=True):
+    """Route every following call to libep_checked.so (flag True) or libep.so.
+    A buffer must be used with the library that created it."""
+    global _use_checked
+    _use_checked = bool(flag)
 
 
 def lib():
-    """The loaded libep.so.  Raises if the library has not been built: there is no
-    fallback implementation."""
-    global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError("libep.so is missing at %s; build it with "
-                           "`python -m combine_ep_layout_12_b200.build`" % LIB_PATH)
-    L = ctypes.CDLL(LIB_PATH)
+    """The loaded libep.so (or libep_checked.so after use_checked()).  Raises if the
+    library has not been built: there is no fallback implementation."""
+    path = LIB_CHECKED_PATH if _use_checked else LIB_PATH
+    L = _libs.get(path)
+    if L is not None:
+        return L
+    if not os.path.exists(path):
+        raise RuntimeError("%s is missing; build it with "
+                           "`python -m combine_ep_layout_12_b200.build`" % path)
+    L = _load(path)
+    _libs[path] = L
+    return L
+
+
+def _load(path):
+    L = ctypes.CDLL(path)
     vp, i = ctypes.c_void_p, ctypes.c_int
     L.ep_buffer_size.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_buffer_sizes)]
     L.ep_buffer_create.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_buffer_ptrs),
@@ -73,7 +91,6 @@ def lib():
         f.restype = i
     L.ep_status_str.argtypes = [i]
     L.ep_status_str.restype = ctypes.c_char_p
-    _lib = L
     return L
 
 

@@ -2,6 +2,11 @@
 
     python -m combine_ep_layout_12_b200.build [--force] [--verbose-ptxas]
 
+Also builds libep_checked.so: the same sources with -DEP_CHECKED, in which every
+row or offset a kernel computes is tested against its array's extent before the
+access (EP_ERRBIT_CHECKED in the error word).  The tests run the GPU parity cases
+against it as well; the benchmark uses libep.so.
+
 No fast-math: IEEE division, denormals kept, and every rounding the results
 depend on is written with explicit _rn intrinsics in the kernels.  The CUDA
 runtime is linked statically, so the library needs only the driver at run time.
@@ -16,6 +21,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libep.so")
+LIB_CHECKED = os.path.join(PKG, "libep_checked.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -57,5 +63,10 @@ def build(force=False, verbose_ptxas=False, quiet=True, out=LIB, extra=()):
     return out
 
 
+def build_checked(force=False, quiet=True):
+    return build(force=force, quiet=quiet, out=LIB_CHECKED, extra=("-DEP_CHECKED",))
+
+
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv, quiet=False)
+    build_checked(force="--force" in sys.argv, quiet=False)

@@ -182,13 +182,13 @@ __device__ __forceinline__ void dispatch_int8_body(const DispatchArgs& a, int t)
         if (degenerate) v = make_uint4(0, 0, 0, 0);
         for (int j = 0; j < a.k; ++j) {
             const int row = s_rows[j];
-            if (row >= 0) st_v4(out + (size_t)row * a.d + 16 * u, v);
+            if (row >= 0 && ep_in_range(row, a.rows, a.err)) st_v4(out + (size_t)row * a.d + 16 * u, v);
         }
     }
     if (STATIC) return;
     if (threadIdx.x < a.k) {
         const int row = s_rows[threadIdx.x];
-        if (row >= 0) a.recv_scale[row] = inv;
+        if (row >= 0 && ep_in_range(row, a.rows, a.err)) a.recv_scale[row] = inv;
     }
     if (threadIdx.x == 0) a.token_scale[t] = inv;
 }
@@ -221,7 +221,7 @@ __device__ __forceinline__ void dispatch_bf16_body(const DispatchArgs& a, int t)
         if (u >= nvec) continue;
         for (int j = 0; j < a.k; ++j) {
             const int row = s_rows[j];
-            if (row >= 0) st_v4(out + (size_t)row * nvec + u, raw[i]);
+            if (row >= 0 && ep_in_range(row, a.rows, a.err)) st_v4(out + (size_t)row * nvec + u, raw[i]);
         }
     }
 }

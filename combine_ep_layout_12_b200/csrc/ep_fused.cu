@@ -85,6 +85,7 @@ int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_
     la.sp_partial = nullptr;
     la.B = s.B; la.k = s.k; la.P = s.P; la.M = s.M; la.E = s.E; la.T = s.T;
     la.n_special = s.n_special; la.E_tot = s.E_tot;
+    la.rows = s.rows;
     la.warps = warps;
     DispatchArgs da = make_dispatch_args(s, p, x, smooth, topk_idx, active);
     da.self_rows = 1;

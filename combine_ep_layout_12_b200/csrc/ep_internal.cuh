@@ -160,6 +160,20 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     return m;
 }
 
+// Checked build (-DEP_CHECKED): every row or offset a kernel computes is tested
+// against the extent of the array it indexes before the access; one outside it
+// sets EP_ERRBIT_CHECKED in the error word and the access is skipped.  Without
+// EP_CHECKED the test compiles away (the kernels' own range checks stay).
+#ifdef EP_CHECKED
+__device__ __forceinline__ bool ep_in_range(long long idx, long long n, unsigned* err_word) {
+    if (idx >= 0 && idx < n) return true;
+    atomicOr(err_word, EP_ERRBIT_CHECKED);
+    return false;
+}
+#else
+__device__ __forceinline__ bool ep_in_range(long long, long long, unsigned*) { return true; }
+#endif
+
 // OR `bits` into the device error word, one atomic per group of converged lanes.
 __device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
     const unsigned active = __activemask();

@@ -128,7 +128,8 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
                     const int g = ids[j];
                     const int slot = my_pre[g] + __popc(my_mask[g] & lt);
                     row = g * a.P * a.M + r * a.M + slot;
-                    if (a.recv_src) a.recv_src[row] = t;
+                    if (!ep_in_range(row, a.rows, &a.ws->err)) row = -1;
+                    else if (a.recv_src) a.recv_src[row] = t;
                 }
                 a.dst_pos[(size_t)t * k + j] = row;
             }
@@ -183,7 +184,7 @@ __global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
 __global__ void __launch_bounds__(256) layout_pack_kernel(const int32_t* expert_offset,
                                                           const int32_t* recv_count, int32_t* dst_pos,
                                                           int32_t* recv_src, int B, int k, int P,
-                                                          int T, int E) {
+                                                          int T, int E, unsigned* err) {
     extern __shared__ int base[];  // [E][P]
     pdl_wait();
     pdl_launch_dependents();
@@ -204,7 +205,15 @@ __global__ void __launch_bounds__(256) layout_pack_kernel(const int32_t* expert_
         const int g = v / PT;
         const int rem = v - g * PT;
         const int r = rem / T;
+        if (!ep_in_range((long long)g * P + r, (long long)E * P, err)) {
+            dst_pos[i] = -1;
+            continue;
+        }
         const int row = base[g * P + r] + (rem - r * T);
+        if (!ep_in_range(row, n, err)) {
+            dst_pos[i] = -1;
+            continue;
+        }
         dst_pos[i] = row;
         recv_src[row] = (int)(i / k);
     }
@@ -239,7 +248,8 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         if (grid < 1) grid = 1;
         cudaError_t e = launch_pdl(layout_pack_kernel, dim3((unsigned)grid), dim3(256), smem, stream,
                                    (const int32_t*)p.expert_offset, (const int32_t*)p.recv_count,
-                                   p.dst_pos, p.recv_src, s.B, s.k, s.P, s.T, s.E);
+                                   p.dst_pos, p.recv_src, s.B, s.k, s.P, s.T, s.E,
+                                   &reinterpret_cast<WsHeader*>(p.workspace)->err);
         return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
     }
     if (s.B == 0) {
@@ -279,6 +289,7 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         a1.sp_partial = nullptr;
         a1.B = s.B; a1.k = s.k; a1.P = s.P; a1.M = s.M; a1.E = s.E; a1.T = s.T;
         a1.n_special = s.n_special; a1.E_tot = s.E_tot;
+        a1.rows = s.rows;
         a1.warps = 8;
         const int ranks_per_cta = 8 / cpr;
         const int grid = 1 + (s.P + ranks_per_cta - 1) / ranks_per_cta;
@@ -330,6 +341,7 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     a.sp_partial = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.workspace) + sizeof(WsHeader));
     a.B = s.B; a.k = s.k; a.P = s.P; a.M = s.M; a.E = s.E; a.T = s.T;
     a.n_special = s.n_special; a.E_tot = s.E_tot;
+    a.rows = s.rows;
     a.warps = warps;
     cudaError_t e;
     if (s.k <= 2)

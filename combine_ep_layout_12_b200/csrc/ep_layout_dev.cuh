@@ -18,6 +18,7 @@ struct LayoutArgs {
     WsHeader* ws;
     int32_t* sp_partial;  // [P][n_special]
     int B, k, P, M, E, T, n_special, E_tot;
+    long long rows;       // receive rows the computed row ids index (E * P * M)
     int warps;            // warps per CTA
 };
 
@@ -213,7 +214,8 @@ __device__ __forceinline__ void layout_small_body(const LayoutArgs& a, int cpr, 
                 int before = 0;  // the rank's tokens in its earlier chunks that routed to g
                 for (int cc = 0; cc < c; ++cc) before += __popc(rank_masks[(size_t)cc * E + g]);
                 row = g * P * a.M + r * a.M + before + __popc(my_mask[g] & lt);
-                if (a.recv_src) a.recv_src[row] = t;
+                if (!ep_in_range(row, a.rows, &a.ws->err)) row = -1;
+                else if (a.recv_src) a.recv_src[row] = t;
             }
             a.dst_pos[(size_t)t * k + j] = row;
         }

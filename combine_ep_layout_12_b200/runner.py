@@ -49,18 +49,21 @@ class Pipeline:
     not part of dispatch/combine).
     """
 
-    def __init__(self, w, device, alias_expert_out=None):
+    def __init__(self, w, device, alias_expert_out=None, alloc=None):
         self.w = w
         self.device = torch.device(device)
-        self.buf = EPBuffer(w, device=self.device)
+        self.buf = EPBuffer(w, device=self.device, alloc=alloc)
+        if alloc is None:
+            def alloc(shape, dtype):
+                return torch.empty(shape, dtype=dtype, device=self.device)
         if alias_expert_out is None:
             alias_expert_out = w.quant_mode == 0
         if alias_expert_out:
             assert w.quant_mode == 0
             self.expert_out = self.buf.recv_x
         else:
-            self.expert_out = torch.empty((w.rows, w.d), dtype=torch.bfloat16, device=self.device)
-        self.y = torch.empty((w.B, w.d), dtype=torch.bfloat16, device=self.device)
+            self.expert_out = alloc((w.rows, w.d), torch.bfloat16)
+        self.y = alloc((w.B, w.d), torch.bfloat16)
 
     def layout(self, dev_inp, stream=None):
         self.buf.layout(dev_inp["topk_idx"], x_active_mask=dev_inp.get("active"), stream=stream)

@@ -101,6 +101,9 @@ typedef struct CUstream_st* ep_stream_t;
 #define EP_ERRBIT_DUP_ID 0x2u /* a routed id repeated in one token: later copies dropped */
 #define EP_ERRBIT_ROW_RANGE 0x4u /* a dst_pos outside [-1, E*P*M) reached dispatch or
                                     combine (e.g. no ep_layout ran): that pick was skipped */
+#define EP_ERRBIT_CHECKED 0x8u /* checked build only (libep_checked.so, -DEP_CHECKED): a
+                                   row or offset a kernel computed fell outside the array it
+                                   indexes; that access was skipped.  Never set by libep.so. */
 
 /*
  * Problem description.  Constraints checked by ep_buffer_size/ep_buffer_create:

@@ -7,6 +7,7 @@ the oracle's layout names, so the GPU combine reads them through its own
 dst_pos.
 """
 import numpy as np
+import pytest
 import torch
 
 import oracle
@@ -181,3 +182,54 @@ def compare_combine(rep, name, y_gpu, y_ref, idx, wts, compact, vals, x, w):
     rep.check(bool(ok.all()), "%s: combine outside tolerance at %d elements" % (name, int((~ok).sum())))
     rep.check(n_diff == 0, "%s: combine not bit-exact at %d elements (within tolerance: %s)"
               % (name, n_diff, bool(ok.all())))
+
+
+def same_as_x(y, x):
+    """y == x bitwise, except that -0 in x must come back as +0 (an exact sum of
+    zeros rounds to +0)."""
+    xi = x.view(torch.int16)
+    want = torch.where(xi == -32768, torch.zeros_like(xi), xi)
+    return torch.equal(y.view(torch.int16), want)
+
+
+def free_bytes():
+    torch.cuda.empty_cache()
+    return torch.cuda.mem_get_info()[0]
+
+
+def need_bytes(w, separate_expert_out):
+    rows = w.rows
+    esz = 1 if w.quant_mode != 0 else 2
+    total = rows * w.d * esz + rows * 4 * (3 if w.quant_mode == 2 else 1)
+    if separate_expert_out:
+        total += rows * w.d * 2
+    total += 2 * w.B * w.d * 2 + 16 * w.B * w.k
+    return total
+
+
+def full_check(w, dev, inp=None, tokens=None, sample_picks=None, separate=True, fused=False,
+               alloc=None):
+    """Layout + dispatch + combine of one workload against the oracle.  fused: issue
+    layout and dispatch as the single ep_layout_dispatch call; alloc: how the
+    device arrays are allocated (see EPBuffer)."""
+    inp = inp if inp is not None else wl.generate(w)
+    if need_bytes(w, separate) > free_bytes() - (4 << 30):
+        pytest.skip("%s needs %.1f GB of device memory" % (w.name, need_bytes(w, separate) / 1e9))
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev, alias_expert_out=not separate, alloc=alloc)
+    rep = Report()
+    if fused:
+        pipe.layout_dispatch(dev_inp)
+    else:
+        pipe.layout(dev_inp)
+        pipe.dispatch(dev_inp)
+    err = pipe.buf.check()
+    ref = oracle.layout(ocfg(w), inp["topk_idx"], active=inp.get("active"))
+    rep.check(err == ref["err"], "%s: device error bits %#x, oracle %#x" % (w.name, err, ref["err"]))
+    check_layout(rep, w, pipe, ref)
+    check_dispatch(rep, w, pipe, inp, ref, sample_picks=sample_picks)
+    check_combine(rep, w, pipe, inp, dev_inp, ref, tokens=tokens)
+    err = pipe.buf.check()
+    rep.check(err == 0, "%s: error bits after combine %#x" % (w.name, err))
+    rep.assert_ok()
+    return pipe, dev_inp, inp, ref

@@ -16,6 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 @pytest.fixture(scope="module", autouse=True)
 def built():
     ep_build.build()
+    ep_build.build_checked()
 
 
 def declared_entry_points():
@@ -27,10 +28,11 @@ def declared_entry_points():
     return names
 
 
-def test_exports_every_declared_symbol():
+@pytest.mark.parametrize("path", [abi.LIB_PATH, abi.LIB_CHECKED_PATH])
+def test_exports_every_declared_symbol(path):
     names = declared_entry_points()
     assert len(names) >= 8
-    lib = ctypes.CDLL(abi.LIB_PATH)
+    lib = ctypes.CDLL(path)
     missing = [n for n in names if not hasattr(lib, n)]
     assert not missing, missing
 
