@@ -112,9 +112,16 @@ class EPBuffer:
             raise ValueError("x_active_mask must be a contiguous [B] tensor on %s" % self.device)
         return _ptr(t)
 
-    def _smooth_shape(self):
+    def _smooth(self, smooth_scale):
+        """Checked pointer of a smooth scale: [d] (or [1, d]) for smooth_rows 1,
+        [smooth_rows, d] per routed expert otherwise; None passes through."""
+        if smooth_scale is None:
+            return None
         c = self.cfg
-        return (c.d,) if c.smooth_rows <= 1 else (c.smooth_rows, c.d)
+        if c.smooth_rows <= 1 and smooth_scale.dim() == 2 and smooth_scale.shape[0] == 1:
+            smooth_scale = smooth_scale[0]
+        shape = (c.d,) if c.smooth_rows <= 1 else (c.smooth_rows, c.d)
+        return _ptr(_need(smooth_scale, "smooth_scale", torch.float32, shape, self.device))
 
     # -- hot path ---------------------------------------------------------------
     def layout(self, topk_idx, x_active_mask=None, stream=None):
@@ -125,19 +132,15 @@ class EPBuffer:
     def dispatch(self, x, smooth_scale=None, stream=None):
         c = self.cfg
         _need(x, "x", torch.bfloat16, (c.B, c.d), self.device)
-        if smooth_scale is not None:
-            _need(smooth_scale, "smooth_scale", torch.float32, self._smooth_shape(), self.device)
-        ep_dispatch(self.handle, _ptr(x), _ptr(smooth_scale), _stream(stream))
+        ep_dispatch(self.handle, _ptr(x), self._smooth(smooth_scale), _stream(stream))
 
     def layout_dispatch(self, topk_idx, x, smooth_scale=None, x_active_mask=None, stream=None):
         """layout(topk_idx) then dispatch(x), as one call (one grid when T <= 128)."""
         c = self.cfg
         _need(topk_idx, "topk_idx", torch.int32, (c.B, c.k), self.device)
         _need(x, "x", torch.bfloat16, (c.B, c.d), self.device)
-        if smooth_scale is not None:
-            _need(smooth_scale, "smooth_scale", torch.float32, self._smooth_shape(), self.device)
         ep_layout_dispatch(self.handle, _ptr(topk_idx), self._mask(x_active_mask), _ptr(x),
-                           _ptr(smooth_scale), _stream(stream))
+                           self._smooth(smooth_scale), _stream(stream))
 
     def combine(self, expert_out, topk_idx, topk_weights, ori_x=None, a1=None, a2=None, v=None,
                 y=None, x_active_mask=None, stream=None):
