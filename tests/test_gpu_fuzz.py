@@ -20,7 +20,7 @@ from tests.test_gpu_checked import Guarded
 
 pytestmark = pytest.mark.gpu
 
-N_CASES = 150
+N_CASES = 300
 
 
 @pytest.fixture(scope="module")
