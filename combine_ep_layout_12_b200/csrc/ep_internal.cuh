@@ -83,14 +83,25 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
 inline int num_sms() {
     static int cached[64] = {0};
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && cached[dev] != 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+// One-time per-device setup (a kernel's shared-memory opt-in is a per-device
+// attribute).  first_on_device is true until mark_device records the device; past
+// the table it stays true, so the setup simply runs on every call there.  Setting
+// the same attribute twice is harmless, so concurrent first calls need no lock.
+constexpr int kDeviceSlots = 64;
+inline bool first_on_device(const bool* done, int dev) {
+    return dev < 0 || dev >= kDeviceSlots || !done[dev];
+}
+inline void mark_device(bool* done, int dev) {
+    if (dev >= 0 && dev < kDeviceSlots) done[dev] = true;
 }
 
 // Launch with programmatic dependent launch enabled: the kernel may begin while

@@ -234,14 +234,14 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         const int st = launch_layout(ll, q, topk_idx, active, stream);
         if (st != EP_OK) return st;
         const size_t smem = sizeof(int) * (size_t)s.E * s.P;
-        static bool attr_pack[64] = {false};
+        static bool attr_pack[kDeviceSlots] = {false};
         int dev = 0;
         cudaGetDevice(&dev);
-        if (dev >= 0 && dev < 64 && !attr_pack[dev]) {
+        if (first_on_device(attr_pack, dev)) {
             if (cudaFuncSetAttribute(layout_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)(sizeof(int) * kMaxPackedEP)) != cudaSuccess)
                 return EP_ERR_CUDA;
-            attr_pack[dev] = true;
+            mark_device(attr_pack, dev);
         }
         long long grid = ((long long)s.B * s.k + 1023) / 1024;
         if (grid > (long long)num_sms() * 4) grid = (long long)num_sms() * 4;
@@ -260,7 +260,7 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         return (e1 || e2 || e3) ? EP_ERR_CUDA : EP_OK;
     }
     const size_t budget = 160 * 1024;
-    static bool attr_small[16] = {false};
+    static bool attr_small[kDeviceSlots] = {false};
     int dev0 = 0;
     cudaGetDevice(&dev0);
     // small per-rank batches: count CTA + slot CTAs, no inter-CTA dependency
@@ -269,13 +269,13 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     const size_t smem_slot = sizeof(int) * (size_t)8 * s.E;
     const size_t smem_small = smem_count > smem_slot ? smem_count : smem_slot;
     if (s.T <= 256 && smem_small <= budget) {
-        if (dev0 < 16 && !attr_small[dev0]) {
+        if (first_on_device(attr_small, dev0)) {
             if (cudaFuncSetAttribute(layout_small_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
                 cudaFuncSetAttribute(layout_small_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
                 cudaFuncSetAttribute(layout_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
                 cudaFuncSetAttribute(layout_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget))
                 return EP_ERR_CUDA;
-            attr_small[dev0] = true;
+            mark_device(attr_small, dev0);
         }
         LayoutArgs a1;
         a1.topk_idx = topk_idx;
@@ -317,16 +317,16 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     if (smem < need_tail) smem = need_tail;
     if (smem > budget) return EP_ERR_UNSUPPORTED;
 
-    static bool attr_set[16] = {false};
+    static bool attr_set[kDeviceSlots] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 16 && !attr_set[dev]) {
+    if (first_on_device(attr_set, dev)) {
         if (cudaFuncSetAttribute(layout_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
             cudaFuncSetAttribute(layout_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
             cudaFuncSetAttribute(layout_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
             cudaFuncSetAttribute(layout_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget))
             return EP_ERR_CUDA;
-        attr_set[dev] = true;
+        mark_device(attr_set, dev);
     }
 
     LayoutArgs a;
@@ -384,7 +384,8 @@ cudaError_t static_scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (dev < 0) return cudaErrorInvalidDevice;
+    if (dev >= kMaxDevices) return cudaGetSymbolAddress(out, g_layout_scratch);  // not cached
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
     if (!g_scratch_addr[dev]) {
         void* p = nullptr;
