@@ -67,6 +67,14 @@
  *    device error word, read by ep_buffer_check.
  *  - The device that runs the kernels is the one current on the calling thread
  *    (the CUDA context current when the call is made).
+ *  - An ep_buffer is not thread-safe: calls on one buffer must not overlap on the
+ *    host, and its kernels must be ordered on one stream (each call reuses the
+ *    buffer's arrays and the routing of its latest layout).  Different buffers
+ *    are independent.
+ *  - Entry points make no device allocation and, apart from ep_buffer_create and
+ *    ep_buffer_check, no synchronizing call, so they can be captured into CUDA
+ *    graphs (make one eager call of each per device first: the first launch of a
+ *    kernel sets its shared-memory opt-in).
  */
 #ifndef EP_H
 #define EP_H
