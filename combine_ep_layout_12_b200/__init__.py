@@ -7,6 +7,23 @@ below is a convenience wrapper that allocates the caller-owned arrays as torch
 tensors and passes their addresses through.  torch supplies device memory and
 streams only.  There is no CPU or torch fallback: every call fails loudly if
 libep.so is missing.
+
+Usage (one decode step of 8 logical ranks x 128 tokens, DeepSeek-V3 shape):
+
+    cfg = make_config(B=1024, d=7168, k=8, P=8, M=128, E=256, quant_mode=2, smooth_rows=1)
+    buf = EPBuffer(cfg, device="cuda")
+    buf.layout_dispatch(topk_idx, x)          # int32 [B, k], bf16 [B, d]
+    # buf.recv_x [E*P*M, d] int8 and buf.recv_scale [E*P*M]: rank q's experts
+    # q*L .. q*L+L-1 own rows [q*L*P*M, (q+1)*L*P*M); buf.recv_count [E, P] counts
+    # them per source rank.  Run the experts, write bf16 outputs to expert_out
+    # at the same rows, then:
+    y = buf.combine(expert_out, topk_idx, topk_weights, ori_x=x)
+
+Options: quant_mode 0 (bf16) / 1 (static int8) / 2 (dynamic int8); smooth_rows
+= E for a per-expert [E, d] smooth scale; layout=1 for rows packed per expert
+(rank q reads [expert_offset[q*L], expert_offset[(q+1)*L])); n_zero / n_copy /
+n_const special experts (combine then needs ori_x, and a1, a2, v for constant
+experts); x_active_mask= on layout / layout_dispatch / combine.
 """
 import torch
 
