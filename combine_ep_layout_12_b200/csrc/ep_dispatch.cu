@@ -323,7 +323,14 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
     DispatchArgs a = make_dispatch_args(s, p, x, smooth, topk_idx, active);
     // Small batches per rank: each CTA derives its rows from the routing itself
     // (at most kSelfRowsMaxT earlier tokens to scan), so dispatch overlaps layout.
-    a.self_rows = (topk_idx != nullptr && s.layout == 0 && s.T <= kSelfRowsMaxT) ? 1 : 0;
+    // Packed rows also need the layout kernel's counts: ep_layout ends with the pack
+    // kernel, which starts only after the counting kernel has finished, so a
+    // dispatch started by the pack kernel can read them and run alongside it.
+    a.self_rows = (topk_idx != nullptr && s.T <= kSelfRowsMaxT) ? 1 : 0;
+    if (a.self_rows && s.layout == 1) {
+        a.expert_offset = p.expert_offset;
+        a.recv_count = p.recv_count;
+    }
     int U = 0, NT = 0;
     cudaError_t e = cudaSuccess;
     const dim3 grid(s.B);

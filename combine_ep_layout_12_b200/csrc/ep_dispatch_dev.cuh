@@ -17,6 +17,8 @@ struct DispatchArgs {
     const int32_t* topk_idx; // [B][k]; read instead of dst_pos when self_rows
     const uint8_t* active;   // x_active_mask [B] or null (self_rows only: dst_pos has it)
     int self_rows;           // compute the receive rows here (small T) instead of reading dst_pos
+    const int32_t* expert_offset;  // packed rows with self_rows: the layout's counts
+    const int32_t* recv_count;
     int T, P, M, E;
     void* recv_x;            // [rows][d] int8 or bf16
     float* recv_scale;       // [rows]
@@ -30,7 +32,8 @@ struct DispatchArgs {
 // while the x row load is in flight.
 __device__ __forceinline__ void compute_rows(const DispatchArgs& a, int t, int* s_rows, int* s_g,
                                              int* s_cnt) {
-    routing_rows(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt);
+    routing_rows(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt,
+                 a.expert_offset, a.recv_count);
 }
 
 // Receive rows of token t into shared memory; out-of-range rows are skipped and flagged.
@@ -245,6 +248,8 @@ inline DispatchArgs make_dispatch_args(const Shape& s, const ep_buffer_ptrs& p, 
     a.k = s.k;
     a.topk_idx = topk_idx;
     a.self_rows = 0;
+    a.expert_offset = nullptr;
+    a.recv_count = nullptr;
     a.T = s.T;
     a.P = s.P;
     a.M = s.M;

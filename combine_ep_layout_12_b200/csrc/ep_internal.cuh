@@ -200,8 +200,14 @@ __device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
 // nothing and are not counted.  The earlier tokens' ids come from L2.  s_rows,
 // s_g, s_cnt: k-entry shared arrays.  All threads of the CTA call it; on return
 // s_rows[j] is written by thread j (j < k) and not yet published to the other threads.
+// Packed rows (expert_offset and recv_count given): the row is expert_offset[g] +
+// sum_{r' < r} recv_count[g][r'] + slot.  Those counts come from the layout kernel,
+// which the caller guarantees complete; they are read through L2 (another grid
+// wrote them).
 __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* active, int t, int k,
-                                    int E, int T, int P, int M, int* s_rows, int* s_g, int* s_cnt) {
+                                    int E, int T, int P, int M, int* s_rows, int* s_g, int* s_cnt,
+                                    const int32_t* expert_offset = nullptr,
+                                    const int32_t* recv_count = nullptr) {
     if (threadIdx.x < k) {
         const int j = threadIdx.x;
         const int g = topk_idx[(size_t)t * k + j];
@@ -230,10 +236,23 @@ __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* acti
             atomicAdd(&s_cnt[j], 1);
         }
     }
+    if (expert_offset) {
+        // packed: add each pick's base (expert_offset[g] and the r lower ranks' counts)
+        // to its slot, all the loads spread over the CTA's threads at once
+        const int per = r + 1;
+        for (int i = threadIdx.x; i < k * per; i += blockDim.x) {
+            const int j = i / per, rr = i - j * per;
+            const int g = s_g[j];
+            if (g >= 0)
+                atomicAdd(&s_cnt[j], rr < r ? __ldcg(recv_count + (size_t)g * P + rr) : __ldcg(expert_offset + g));
+        }
+    }
     __syncthreads();
     if (threadIdx.x < k) {
         const int g = s_g[threadIdx.x];
-        s_rows[threadIdx.x] = g >= 0 ? g * P * M + r * M + s_cnt[threadIdx.x] : -1;
+        int row = -1;
+        if (g >= 0) row = expert_offset ? s_cnt[threadIdx.x] : g * P * M + r * M + s_cnt[threadIdx.x];
+        s_rows[threadIdx.x] = row;
     }
 }
 
