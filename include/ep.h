@@ -210,8 +210,9 @@ EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, const uint8_t* x_a
  * receive row whose recv_src is not a token sets EP_ERRBIT_ROW_RANGE and is skipped.
  * For T = B/P <= 256 the kernel derives those rows from the topk_idx (and mask)
  * passed to that ep_layout (which must still hold the same values) instead of reading dst_pos,
- * so it can run alongside the layout kernel; it finishes only after the layout
- * kernel has.  Call it on the stream of that ep_layout, after it. */
+ * so it can run alongside the layout kernel (for the packed layout, alongside its
+ * second kernel, reading the per-expert counts the first one wrote); it finishes
+ * only after the layout kernels have.  Call it on the stream of that ep_layout, after it. */
 EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale,
                 ep_stream_t stream);
 
@@ -231,7 +232,9 @@ EP_API int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx,
  * x_active_mask uint8 [B] or NULL, the mask given to ep_layout (inactive tokens
  * get y = +0);
  * ori_x bf16 [B][d] (required when C + K > 0, else may be NULL);
- * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos.
+ * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos,
+ * or for T = B/P <= 128 derives the same rows from topk_idx (which must hold the
+ * ids given to that layout) and the layout's counts.
  * y must not overlap any input. */
 EP_API int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,
                const float* topk_weights, const uint8_t* x_active_mask, const uint16_t* ori_x,
