@@ -82,7 +82,8 @@ int launch_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_
     la.dst_pos = p.dst_pos;
     la.recv_src = p.recv_src;
     la.ws = reinterpret_cast<WsHeader*>(p.workspace);
-    la.sp_partial = nullptr;
+    la.chunk_cnt = nullptr;
+    la.sp_chunk = nullptr;
     la.B = s.B; la.k = s.k; la.P = s.P; la.M = s.M; la.E = s.E; la.T = s.T;
     la.n_special = s.n_special; la.E_tot = s.E_tot;
     la.rows = s.rows;

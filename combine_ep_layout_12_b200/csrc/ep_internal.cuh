@@ -48,10 +48,12 @@ inline Shape make_shape(const ep_config& c) {
     return s;
 }
 
-// Workspace layout: WsHeader, then the multi-CTA layout's per-rank special
-// counts [P][n_special].
+// Workspace layout: WsHeader, then, for batches of more than 256 tokens per rank
+// (the chunked layout kernels), the per-chunk counts [P][chunks][E] and special
+// counts [P][chunks][n_special], chunks = ceil(T / 256).
 inline size_t workspace_layout_bytes(const Shape& s) {
-    return sizeof(WsHeader) + 4 * (size_t)s.P * s.n_special;
+    const size_t chunks = s.T > 256 ? ((size_t)s.T + 255) / 256 : 0;
+    return sizeof(WsHeader) + 4 * (size_t)s.P * chunks * ((size_t)s.E + s.n_special);
 }
 inline size_t workspace_bytes(const Shape& s) {
     return (workspace_layout_bytes(s) + 255) & ~(size_t)255;

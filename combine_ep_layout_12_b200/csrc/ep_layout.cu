@@ -7,17 +7,15 @@
 // deterministic computation).  Expert g lives on rank g / (E / P) (DeepEP issue
 // #84, masking experiment); id -1 sends nothing.
 //
-// Design.  One CTA per source rank r.  The rank's tokens are processed in rounds
-// of (warps x 32) tokens, one token per lane.  In a round every warp builds, in
-// shared memory, a 32-bit lane mask per routed expert (atomicOr of bit `lane`
-// for each of its token's routed ids).  Because OR is order-independent the
-// masks, and everything derived from them, are deterministic.  An exclusive scan
-// over the warps of popc(mask) per expert, plus the counts of earlier rounds,
-// gives each warp's base; a token's slot inside its (expert, rank) run is then
-//     base[w][g] + popc(mask[w][g] & lanemask_lt)
-// i.e. its rank among rank r's tokens that routed to g, in ascending token order.
-// The last CTA to finish (a ticket counter in the workspace; no CTA ever waits on
-// another) adds the per-rank counts into expert_count and scans expert_offset.
+// Design.  Every variant builds, in shared memory, one 32-bit lane mask per
+// routed expert for each warp's 32 tokens (atomicOr of bit `lane` for each of the
+// token's routed ids).  OR is order-independent, so the masks and everything
+// derived from them are deterministic.  A token's slot inside its (expert, rank)
+// run is the count of the rank's earlier tokens that picked g plus
+// popc(mask[w][g] & lanemask_lt), i.e. its rank among rank r's tokens that routed
+// to g, in ascending token order.  Batches of up to 256 tokens per rank use one
+// kernel (ep_layout_dev.cuh); larger ones two kernels over 256-token chunks, below.
+// No CTA ever waits on another.
 #include <mutex>
 
 #include "ep_internal.cuh"
@@ -34,144 +32,144 @@ __global__ void __launch_bounds__(256) layout_small_kernel(LayoutArgs a, int cpr
     layout_small_body<KM>(a, cpr, blockIdx.x, smem);
 }
 
+// Layout for larger per-rank batches (T > 256), in two kernels over (chunk, rank)
+// CTAs, a chunk being 256 consecutive tokens of one rank; no CTA ever waits on
+// another.
+//  - Count kernel: each CTA builds the lane masks of its chunk (one warp per 32
+//    tokens, as in the small-batch layout), writes the chunk's routed picks per
+//    expert and its special-expert counts to the workspace, and leaves each routed
+//    pick's slot within the chunk in dst_pos.
+//  - Rows kernel: each CTA sums the counts of its rank's earlier chunks per expert
+//    (all the loads spread over the CTA at once) and turns the in-chunk slots into
+//    receive rows; the rank's last chunk also writes recv_count.  The last CTA to
+//    finish (a ticket counter) adds the counts over ranks into expert_count and
+//    scans expert_offset.
+// Slots stay in ascending token order: the earlier chunks' counts come first, then
+// the lane-mask rank inside the chunk.
+constexpr int kChunkTokens = 256;
+
 template <int KM>
-__global__ void __launch_bounds__(1024) layout_kernel(LayoutArgs a) {
+__global__ void __launch_bounds__(kChunkTokens) layout_chunk_count_kernel(LayoutArgs a, int n_chunks) {
     extern __shared__ unsigned smem[];
-    const int W = a.warps;
-    unsigned* mask = smem;                                         // [W][E]
-    int* pre = reinterpret_cast<int*>(smem + (size_t)W * a.E);     // [W][E]
-    int* run = pre + (size_t)W * a.E;                              // [E] count so far
-    int* spc = run + a.E;                                          // [n_special]
-    __shared__ int s_last;
-
-    const int r = blockIdx.x;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
     const int E = a.E, k = a.k;
-
+    constexpr int W = kChunkTokens / 32;
+    unsigned* mask = smem;                                     // [W][E]
+    int* spc = reinterpret_cast<int*>(smem + (size_t)W * E);  // [n_special]
     pdl_wait();
     pdl_launch_dependents();
-
-    for (int g = threadIdx.x; g < E; g += blockDim.x) run[g] = 0;
-    for (int s = threadIdx.x; s < a.n_special; s += blockDim.x) spc[s] = 0;
-
-    unsigned err = 0;
-    const int tok_begin = r * a.T;
-    const int tok_end = tok_begin + a.T;
-    const int per_round = W * 32;
-    unsigned* my_mask = mask + (size_t)warp * E;
-    int* my_pre = pre + (size_t)warp * E;
-
-    for (int round0 = tok_begin; round0 < tok_end; round0 += per_round) {
-        // (1) clear this warp's masks (the previous round's readers of my_mask
-        //     are this warp's own lanes, so a warp barrier suffices)
-        __syncwarp();
-        for (int g = lane; g < E; g += 32) my_mask[g] = 0u;
-        __syncthreads();  // also orders run[] / spc[] init before first use
-
-        const int t = round0 + warp * 32 + lane;
-        const bool valid = t < tok_end;
-        int ids[KM];
-        bool routed[KM];
-        const bool on = valid && !(a.active && !a.active[t]);  // x_active_mask
+    const int c = blockIdx.x, r = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i < W * E; i += blockDim.x) mask[i] = 0u;
+    for (int i = threadIdx.x; i < a.n_special; i += blockDim.x) spc[i] = 0;
+    __syncthreads();
+    const int tr = c * kChunkTokens + (int)threadIdx.x;  // token index inside the rank
+    const bool valid = tr < a.T;
+    const int t = r * a.T + tr;
+    const bool vec4 = (k % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.topk_idx) & 15) == 0);
+    int ids[KM];
+    unsigned rb = 0, err = 0;
+    if (valid) {
+        load_token_ids<KM>(a.topk_idx, t, k, vec4, ids);
+        apply_active<KM>(a.active, t, ids);
+        rb = classify_ids<KM>(ids, k, E, a.E_tot, err, [&](int sidx) { atomicAdd(&spc[sidx], 1); });
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+        if (rb & (1u << j)) atomicOr(&mask[(size_t)warp * E + ids[j]], 1u << lane);
+    __syncthreads();
+    if (valid) {
+        const unsigned lt = lanemask_lt();
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
-            ids[j] = -1;
-            routed[j] = false;
-            if (j < k && on) ids[j] = a.topk_idx[(size_t)t * k + j];
-        }
-        // (2) classify; routed ids set their lane bit
-#pragma unroll
-        for (int j = 0; j < KM; ++j) {
-            if (j >= k || !valid) continue;
-            const int g = ids[j];
-            if (g == -1) continue;
-            if (g < -1 || g >= a.E_tot) {
-                err |= EP_ERRBIT_BAD_ID;
-                continue;
+            if (j >= k) continue;
+            int slot = -1;
+            if (rb & (1u << j)) {
+                const int g = ids[j];
+                slot = __popc(mask[(size_t)warp * E + g] & lt);
+                for (int w = 0; w < warp; ++w) slot += __popc(mask[(size_t)w * E + g]);
             }
-            if (g >= E) {
-                atomicAdd(&spc[g - E], 1);
-                continue;
-            }
-            bool dup = false;
-#pragma unroll
-            for (int jj = 0; jj < KM; ++jj)
-                if (jj < j && ids[jj] == g) dup = true;
-            if (dup) {
-                err |= EP_ERRBIT_DUP_ID;
-                continue;
-            }
-            routed[j] = true;
-            atomicOr(&my_mask[g], 1u << lane);
-        }
-        __syncthreads();
-        // (3) per expert: exclusive scan of the warps' popcounts, on top of the
-        //     counts of earlier rounds
-        for (int g = threadIdx.x; g < E; g += blockDim.x) {
-            int c = run[g];
-            for (int w = 0; w < W; ++w) {
-                pre[(size_t)w * E + g] = c;
-                c += __popc(mask[(size_t)w * E + g]);
-            }
-            run[g] = c;
-        }
-        __syncthreads();
-        // (4) slots, receive rows, source map
-        if (valid) {
-            const unsigned lt = lanemask_lt();
-#pragma unroll
-            for (int j = 0; j < KM; ++j) {
-                if (j >= k) continue;
-                int row = -1;
-                if (routed[j]) {
-                    const int g = ids[j];
-                    const int slot = my_pre[g] + __popc(my_mask[g] & lt);
-                    row = g * a.P * a.M + r * a.M + slot;
-                    if (!ep_in_range(row, a.rows, &a.ws->err)) row = -1;
-                    else if (a.recv_src) a.recv_src[row] = t;
-                }
-                a.dst_pos[(size_t)t * k + j] = row;
-            }
+            a.dst_pos[(size_t)t * k + j] = slot;  // in-chunk slot; the rows kernel adds the rest
         }
     }
-    __syncthreads();
-
-    // per-rank outputs
-    for (int g = threadIdx.x; g < E; g += blockDim.x) a.recv_count[(size_t)g * a.P + r] = run[g];
-    for (int s = threadIdx.x; s < a.n_special; s += blockDim.x)
-        a.sp_partial[(size_t)r * a.n_special + s] = spc[s];
+    int32_t* cnt = a.chunk_cnt + ((size_t)r * n_chunks + c) * E;
+    for (int g = threadIdx.x; g < E; g += blockDim.x) {
+        int n = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) n += __popc(mask[(size_t)w * E + g]);
+        cnt[g] = n;
+    }
+    int32_t* sp = a.sp_chunk + ((size_t)r * n_chunks + c) * a.n_special;
+    for (int i = threadIdx.x; i < a.n_special; i += blockDim.x) sp[i] = spc[i];
     report_err(&a.ws->err, err);
+}
 
-    // ticket: the last CTA of this launch reduces over ranks
+template <int KM>
+__global__ void __launch_bounds__(kChunkTokens) layout_chunk_rows_kernel(LayoutArgs a, int n_chunks) {
+    extern __shared__ int pre[];  // [max(E, E_tot) + 32]: earlier chunks' counts, later the totals
+    __shared__ int s_last;
+    const int E = a.E, k = a.k;
+    pdl_wait();
+    pdl_launch_dependents();
+    const int c = blockIdx.x, r = blockIdx.y;
+    for (int g = threadIdx.x; g < E; g += blockDim.x) pre[g] = 0;
+    __syncthreads();
+    // the rank's picks per expert in chunks 0..c-1 (the rank's last chunk adds its own
+    // to get recv_count); the loads of all (chunk, expert) pairs are spread at once
+    const int32_t* cnt_r = a.chunk_cnt + (size_t)r * n_chunks * E;
+    const int upto = (c == n_chunks - 1) ? c + 1 : c;
+    for (int i = threadIdx.x; i < upto * E; i += blockDim.x) {
+        const int cc = i / E, g = i - cc * E;
+        if (cc < c) atomicAdd(&pre[g], __ldcg(cnt_r + i));
+    }
+    __syncthreads();
+    if (c == n_chunks - 1) {
+        const int32_t* own = cnt_r + (size_t)c * E;
+        for (int g = threadIdx.x; g < E; g += blockDim.x)
+            a.recv_count[(size_t)g * a.P + r] = pre[g] + __ldcg(own + g);
+    }
+    const int tr = c * kChunkTokens + (int)threadIdx.x;
+    if (tr < a.T) {
+        const int t = r * a.T + tr;
+        const bool vec4 = (k % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.topk_idx) & 15) == 0);
+        int ids[KM];
+        load_token_ids<KM>(a.topk_idx, t, k, vec4, ids);
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            if (j >= k) continue;
+            const int slot = __ldcg(a.dst_pos + (size_t)t * k + j);
+            if (slot < 0) continue;  // not routed (the count kernel left -1)
+            const int g = ids[j];
+            int row = -1;
+            if (ep_in_range(g, E, &a.ws->err)) {
+                row = g * a.P * a.M + r * a.M + pre[g] + slot;
+                if (!ep_in_range(row, a.rows, &a.ws->err)) row = -1;
+                else if (a.recv_src) a.recv_src[row] = t;
+            }
+            a.dst_pos[(size_t)t * k + j] = row;
+        }
+    }
+
+    // ticket: the last CTA of this launch reduces over ranks and scans
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
         const unsigned ticket = atomicAdd(&a.ws->done, 1u);
-        s_last = (ticket == (unsigned)a.P - 1u);
+        s_last = (ticket == gridDim.x * gridDim.y - 1u);
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-
-    // expert_count over all ids, then its exclusive prefix into expert_offset.
-    // The rank loop is unrolled so a thread's loads are in flight together.
-    int* ec = reinterpret_cast<int*>(smem);            // reuse: [E_tot]
-    int* wsum = ec + a.E_tot;                          // [32]
-    for (int g = threadIdx.x; g < a.E_tot; g += blockDim.x) {
-        int v = 0;
-        if (g < E) {
-            const int32_t* src = a.recv_count + (size_t)g * a.P;
-#pragma unroll 8
-            for (int q = 0; q < a.P; ++q) v += __ldcg(src + q);
-        } else {
-#pragma unroll 8
-            for (int q = 0; q < a.P; ++q) v += __ldcg(&a.sp_partial[(size_t)q * a.n_special + (g - E)]);
-        }
-        ec[g] = v;
-        a.expert_count[g] = v;
-    }
+    int* ec = pre;                 // [E_tot]
+    int* wsum = pre + a.E_tot;     // [32]
+    for (int g = threadIdx.x; g < a.E_tot; g += blockDim.x) ec[g] = 0;
     __syncthreads();
+    // totals per expert id: recv_count [E][P] and the chunks' special counts
+    // [P][chunks][n_special], both read contiguously with every load in flight at once
+    for (int i = threadIdx.x; i < E * a.P; i += blockDim.x) atomicAdd(&ec[i / a.P], __ldcg(a.recv_count + i));
+    const int n_sp = a.P * n_chunks * a.n_special;
+    for (int i = threadIdx.x; i < n_sp; i += blockDim.x) atomicAdd(&ec[E + i % a.n_special], __ldcg(a.sp_chunk + i));
+    __syncthreads();
+    for (int g = threadIdx.x; g < a.E_tot; g += blockDim.x) a.expert_count[g] = ec[g];
     block_exclusive_scan(ec, a.E_tot, a.expert_offset, wsum);
     if (threadIdx.x == 0) a.ws->done = 0u;  // re-arm the ticket for the next launch
 }
@@ -286,7 +284,8 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         a1.dst_pos = p.dst_pos;
         a1.recv_src = p.recv_src;
         a1.ws = reinterpret_cast<WsHeader*>(p.workspace);
-        a1.sp_partial = nullptr;
+        a1.chunk_cnt = nullptr;
+        a1.sp_chunk = nullptr;
         a1.B = s.B; a1.k = s.k; a1.P = s.P; a1.M = s.M; a1.E = s.E; a1.T = s.T;
         a1.n_special = s.n_special; a1.E_tot = s.E_tot;
         a1.rows = s.rows;
@@ -304,29 +303,19 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
             e = launch_pdl(layout_small_kernel<16>, dim3(grid), dim3(256), smem_small, stream, a1, cpr);
         return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
     }
-    // multi-CTA path: one CTA per rank; warps per CTA enough for one round of the
-    // rank's tokens, at most 32, within the shared-memory budget (two [warps][E]
-    // arrays plus [E] + specials)
-    const size_t fixed = sizeof(int) * ((size_t)s.E + s.n_special);
-    int warps = (s.T + 31) / 32;
-    if (warps > 32) warps = 32;
-    if (warps < 1) warps = 1;
-    while (warps > 1 && fixed + (size_t)warps * s.E * 8 > budget) --warps;
-    size_t smem = fixed + (size_t)warps * s.E * 8;
-    const size_t need_tail = sizeof(int) * ((size_t)s.E_tot + 32);  // counts + scan of the last CTA
-    if (smem < need_tail) smem = need_tail;
-    if (smem > budget) return EP_ERR_UNSUPPORTED;
-
-    static bool attr_set[kDeviceSlots] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (first_on_device(attr_set, dev)) {
-        if (cudaFuncSetAttribute(layout_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
-            cudaFuncSetAttribute(layout_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
-            cudaFuncSetAttribute(layout_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
-            cudaFuncSetAttribute(layout_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget))
+    // larger batches: the chunked count and rows kernels
+    const int n_chunks = (s.T + kChunkTokens - 1) / kChunkTokens;
+    const size_t smem_count_k = sizeof(unsigned) * (size_t)(kChunkTokens / 32) * s.E + sizeof(int) * s.n_special;
+    const size_t smem_rows_k = sizeof(int) * (((size_t)s.E > (size_t)s.E_tot ? s.E : s.E_tot) + 32);
+    if (smem_count_k > budget || smem_rows_k > budget) return EP_ERR_UNSUPPORTED;
+    static bool attr_chunk[kDeviceSlots] = {false};
+    if (first_on_device(attr_chunk, dev0)) {
+        if (cudaFuncSetAttribute(layout_chunk_count_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+            cudaFuncSetAttribute(layout_chunk_count_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+            cudaFuncSetAttribute(layout_chunk_count_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget) ||
+            cudaFuncSetAttribute(layout_chunk_count_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)budget))
             return EP_ERR_CUDA;
-        mark_device(attr_set, dev);
+        mark_device(attr_chunk, dev0);
     }
 
     LayoutArgs a;
@@ -338,20 +327,32 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     a.dst_pos = p.dst_pos;
     a.recv_src = p.recv_src;
     a.ws = reinterpret_cast<WsHeader*>(p.workspace);
-    a.sp_partial = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.workspace) + sizeof(WsHeader));
+    int32_t* words = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p.workspace) + sizeof(WsHeader));
+    a.chunk_cnt = words;                                                   // [P][n_chunks][E]
+    a.sp_chunk = words + (size_t)s.P * n_chunks * s.E;                     // [P][n_chunks][n_special]
     a.B = s.B; a.k = s.k; a.P = s.P; a.M = s.M; a.E = s.E; a.T = s.T;
     a.n_special = s.n_special; a.E_tot = s.E_tot;
     a.rows = s.rows;
-    a.warps = warps;
+    a.warps = kChunkTokens / 32;
+    const dim3 grid((unsigned)n_chunks, (unsigned)s.P), block(kChunkTokens);
     cudaError_t e;
     if (s.k <= 2)
-        e = launch_pdl(layout_kernel<2>, dim3(s.P), dim3(warps * 32), smem, stream, a);
+        e = launch_pdl(layout_chunk_count_kernel<2>, grid, block, smem_count_k, stream, a, n_chunks);
     else if (s.k <= 4)
-        e = launch_pdl(layout_kernel<4>, dim3(s.P), dim3(warps * 32), smem, stream, a);
+        e = launch_pdl(layout_chunk_count_kernel<4>, grid, block, smem_count_k, stream, a, n_chunks);
     else if (s.k <= 8)
-        e = launch_pdl(layout_kernel<8>, dim3(s.P), dim3(warps * 32), smem, stream, a);
+        e = launch_pdl(layout_chunk_count_kernel<8>, grid, block, smem_count_k, stream, a, n_chunks);
     else
-        e = launch_pdl(layout_kernel<16>, dim3(s.P), dim3(warps * 32), smem, stream, a);
+        e = launch_pdl(layout_chunk_count_kernel<16>, grid, block, smem_count_k, stream, a, n_chunks);
+    if (e != cudaSuccess) return EP_ERR_CUDA;
+    if (s.k <= 2)
+        e = launch_pdl(layout_chunk_rows_kernel<2>, grid, block, smem_rows_k, stream, a, n_chunks);
+    else if (s.k <= 4)
+        e = launch_pdl(layout_chunk_rows_kernel<4>, grid, block, smem_rows_k, stream, a, n_chunks);
+    else if (s.k <= 8)
+        e = launch_pdl(layout_chunk_rows_kernel<8>, grid, block, smem_rows_k, stream, a, n_chunks);
+    else
+        e = launch_pdl(layout_chunk_rows_kernel<16>, grid, block, smem_rows_k, stream, a, n_chunks);
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
 }
 

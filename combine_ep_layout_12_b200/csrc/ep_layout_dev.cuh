@@ -16,7 +16,8 @@ struct LayoutArgs {
     int32_t* dst_pos;
     int32_t* recv_src;
     WsHeader* ws;
-    int32_t* sp_partial;  // [P][n_special]
+    int32_t* chunk_cnt;   // larger batches: [P][chunks][E] routed picks per expert and chunk
+    int32_t* sp_chunk;    // larger batches: [P][chunks][n_special] special-expert picks
     int B, k, P, M, E, T, n_special, E_tot;
     long long rows;       // receive rows the computed row ids index (E * P * M)
     int warps;            // warps per CTA

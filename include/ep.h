@@ -256,8 +256,10 @@ EP_API int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t*
  *
  * Its scratch is a 64 KiB array in the library's static device memory, present
  * on every GPU that loads the library until the process exits.  It holds a
- * 256-byte header plus one int32 per (rank, special expert), so configurations
- * with P * (Z + C + K) > 16320 are rejected with EP_ERR_CAPACITY.
+ * 256-byte header and, for batches of more than 256 tokens per rank, one int32
+ * per (rank, 256-token chunk, expert id): configurations that need more, i.e.
+ * P * ceil(T / 256) * (E + Z + C + K) > 16320 with T > 256, are rejected with
+ * EP_ERR_CAPACITY.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.

@@ -92,11 +92,18 @@ def test_static_scratch_layout_matches_ep_layout(dev, name):
 
 
 def test_static_scratch_refuses_configs_beyond_its_array(dev):
-    # P * (Z + C + K) int32 counts must fit next to the 256-byte header in 64 KiB
-    w = wl.Workload("too_many_specials", B=16, d=16, k=2, P=16, M=1, E=16, n_zero=1100,
-                    quant_mode=0)
+    # above 256 tokens per rank the chunked layout keeps P * ceil(T / 256) * (E + Z + C + K)
+    # int32 counts next to the 256-byte header; 8 * 16 * 256 of them exceed 64 KiB
+    w = wl.Workload("too_many_chunks", B=8 * 4096, d=16, k=2, P=8, M=4096, E=256, quant_mode=0)
     out = _outputs(w, dev)
     idx = torch.zeros((w.B, w.k), dtype=torch.int32, device=dev)
     with pytest.raises(abi.EPError) as ei:
         _static_layout(w, idx, out, torch.cuda.current_stream(dev))
     assert ei.value.status == abi.EP_ERR_CAPACITY
+    # small batches need only the header, whatever the number of special experts
+    w2 = wl.Workload("many_specials", B=16, d=16, k=2, P=16, M=1, E=16, n_zero=1100, quant_mode=0)
+    out2 = _outputs(w2, dev)
+    idx2 = torch.zeros((w2.B, w2.k), dtype=torch.int32, device=dev)
+    _static_layout(w2, idx2, out2, torch.cuda.current_stream(dev))
+    torch.cuda.synchronize(dev)
+    assert int(out2["expert_count"][0].item()) == w2.B  # every pick is expert 0, once per token
