@@ -1,0 +1,40 @@
+"""Host-side pieces of bench.py (CPU only): the latency/bandwidth fit, the
+recorded-traffic lookup and its staleness rule, and the seeded inputs the
+measurements are taken on."""
+import json
+
+import numpy as np
+
+import bench
+from combine_ep_layout_12_b200 import workloads as wl
+
+
+def test_fit_recovers_latency_and_bandwidth():
+    L, bw = 7.5e-6, 6.2e12
+    pts = [(v, L + v / bw) for v in (1e5, 1e6, 1e7, 1e8, 1e9)]
+    f = bench.fit_latency_bandwidth(pts)
+    assert abs(f["L_us"] - 7.5) < 1e-6
+    assert abs(f["BW_eff_gbs"] - 6200.0) < 1e-6
+
+
+def test_recorded_traffic_follows_the_source(tmp_path, monkeypatch):
+    doc = {"w": {"combine": {"dram_bytes_per_launch": 123.0, "source_sha": bench.source_hash("combine")},
+                 "dispatch": {"dram_bytes_per_launch": 45.0, "source_sha": "0" * 16}}}
+    (tmp_path / "traffic.json").write_text(json.dumps(doc))
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    assert bench.recorded_traffic("w", "combine") == 123.0
+    assert bench.recorded_traffic("w", "dispatch") is None      # taken on other kernel source
+    assert bench.recorded_traffic("other", "combine") is None
+
+
+def test_seeded_inputs_are_fixed():
+    """The decode inputs every measurement and parity case uses do not drift."""
+    inp = wl.generate(wl.get("decode"))
+    again = wl.generate(wl.get("decode"))
+    assert np.array_equal(inp["x"], again["x"]) and np.array_equal(inp["topk_idx"], again["topk_idx"])
+    # every token has k distinct routed experts
+    idx = inp["topk_idx"]
+    assert idx.min() >= 0 and idx.max() < 256
+    assert all(len(set(r)) == 8 for r in idx[:64].tolist())
+    w = inp["topk_weights"]
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-6) and (w > 0).all()
