@@ -359,8 +359,8 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
 // ---------------------------------------------------------------------------
 // ep_layout_static_scratch: the layout for callers that cannot allocate.
 //
-// The regular entry point keeps its scratch (ticket counter, error word, per-rank
-// special-expert counts) in a workspace the caller allocates.  Some callers have
+// The regular entry point keeps its scratch (ticket counter, error word, and the
+// chunked layout's per-chunk counts) in a workspace the caller allocates.  Some callers have
 // no way to do that: a serving engine that has already handed every byte of the
 // GPU to its own pool, code that must not call cudaMalloc because it can
 // synchronize the whole device and stall other streams, or a plain C host without

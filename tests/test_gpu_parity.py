@@ -301,7 +301,7 @@ def test_static_quant_closed_forms(dev):
     ("tiny_active", dict(base="tiny_q2", active_frac=0.5)),
     ("decode_active", dict()),                                          # T = 128, one grid
     ("decode_active_bf16", dict(base="decode", quant_mode=0, active_frac=0.75)),
-    ("skewed_active", dict(base="skewed", active_frac=0.6)),            # multi-CTA layout, specials
+    ("skewed_active", dict(base="skewed", active_frac=0.6)),            # chunked layout, specials
     ("decode_active_packed", dict(base="decode", active_frac=0.75, layout=1)),
     ("sweep_T256_active", dict(base="sweep_T256_q2", active_frac=0.8)),
     ("decode_active_expert", dict(base="decode", active_frac=0.75, smooth="expert")),
@@ -455,7 +455,7 @@ def test_max_experts(dev):
 
 
 def test_many_rounds(dev):
-    """2500 tokens per rank: the layout kernel loops over three rounds of 1024."""
+    """2500 tokens per rank: ten 256-token chunks per rank, the last one ragged."""
     w = wl.Workload("rounds", B=2 * 2500, d=32, k=6, P=2, M=2600, E=64, quant_mode=2, seed=12)
     full_check(w, dev)
 
