@@ -543,3 +543,41 @@ def test_roundtrip_identity_decode_shape_bf16(dev):
     dev_inp["topk_weights"] = torch.from_numpy(onehot).to(dev)
     y = pipe.step(dev_inp)
     assert same_as_x(y, dev_inp["x"])
+
+
+# ----------------------------------------------------------------------------- boundaries of the paths
+
+
+@pytest.mark.parametrize("kw", [dict(layout=1), dict(quant_mode=1, smooth="rand"),
+                                dict(smooth="expert"), dict(layout=1, smooth="expert")],
+                         ids=["packed", "static", "expert", "packed_expert"])
+def test_empty_batch_variants(dev, kw):
+    w = small("empty_v", B=0, **kw)
+    buf = EPBuffer(w, device=dev)
+    idx = torch.empty((0, w.k), dtype=torch.int32, device=dev)
+    x = torch.empty((0, w.d), dtype=torch.bfloat16, device=dev)
+    wts = torch.empty((0, w.k), dtype=torch.float32, device=dev)
+    eo = torch.zeros((w.rows, w.d), dtype=torch.bfloat16, device=dev)
+    sm = None
+    if w.smooth == "rand":
+        sm = torch.ones(w.d, dtype=torch.float32, device=dev)
+    elif w.smooth == "expert":
+        sm = torch.ones((w.E, w.d), dtype=torch.float32, device=dev)
+    buf.layout(idx)
+    buf.dispatch(x, sm)
+    y = buf.combine(eo, idx, wts, ori_x=x)
+    assert buf.check() == 0
+    assert y.shape == (0, w.d)
+    assert int(buf.expert_count.sum()) == 0 and int(buf.expert_offset[-1]) == 0
+
+
+@pytest.mark.parametrize("T", [257, 512])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_chunk_boundaries(dev, T, layout):
+    """Tokens per rank just past one 256-token chunk (a one-token last chunk) and
+    exactly two chunks, with special experts, a mask and both layouts."""
+    w = wl.Workload("chunks_T%d_l%d" % (T, layout), B=3 * T, d=64, k=5, P=3, M=T + 3, E=12,
+                    n_zero=1, n_copy=1, n_const=1, quant_mode=2, routing="zipf", zipf_s=0.8,
+                    seed=T + layout, layout=layout, active_frac=0.9)
+    full_check(w, dev)
+    full_check(w.with_(name=w.name + "_fused"), dev, fused=True)
