@@ -421,6 +421,50 @@ class Workbench:
         b.synchronize()
         return a.elapsed_time(b)
 
+    def read_flush(self):
+        """Read a buffer three times the L2 size (one reduction kernel): afterwards
+        L2 holds only clean lines of that buffer, so the next kernel reads its inputs
+        from DRAM and its writes evict nothing that needs writing back, as under a
+        profiler's cache flush.  Not launched with a programmatic edge, so the next
+        kernel cannot start before it has finished."""
+        import torch
+        if self._rf_src is None:
+            self._rf_src = torch.ones(self.READ_FLUSH_BYTES // 4, dtype=torch.float32, device=self.device)
+            self._rf_out = torch.zeros((), dtype=torch.float32, device=self.device)
+        torch.sum(self._rf_src, dim=0, out=self._rf_out)
+
+    READ_FLUSH_BYTES = 384 << 20
+    _rf_src = None
+    _rf_out = None
+
+    def isolated_times(self, reps, keys=("layout", "dispatch", "combine", "layout_dispatch")):
+        """Per-launch milliseconds of each kernel run in isolation: every launch is
+        preceded by read_flush(), so it starts on a clean L2 with its inputs in DRAM
+        and overlaps no other launch of the library; graphs of S such pairs are
+        replayed, and the same graph with the reads alone is timed and subtracted."""
+        def graph(names):
+            def body():
+                for i in range(self.S):
+                    p, d = self.sets[i % self.R]
+                    self.read_flush()
+                    for name in names:
+                        getattr(p, name)(d, self.stream)
+            return self.capture(body)
+        n = max(1, reps // self.S)
+        fg = graph(())
+        self.replay(fg, 1)
+        out = {}
+        for key in keys:
+            g = graph([key])
+            self.replay(g, 1)
+            # alternate kernel and flush-only replays so clock drift hits both alike
+            tk, tf = [], []
+            for _ in range(3):
+                tk.append(self.replay(g, n) / (n * self.S))
+                tf.append(self.replay(fg, n) / (n * self.S))
+            out[key] = statistics.median(tk) - statistics.median(tf)
+        return out, n
+
     def kernel_times(self, launches):
         """Per-launch milliseconds of each kernel and of the one-call layout+dispatch,
         from graphs of S back-to-back launches replayed about `launches / S` times.

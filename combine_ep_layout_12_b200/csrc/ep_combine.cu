@@ -49,6 +49,7 @@ struct CombineArgs {
     const int32_t* expert_offset;  // packed rows with self_rows: the layout's counts
     const int32_t* recv_count;
     int T, P, M;
+    int B;                       // tokens
 };
 
 __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
@@ -163,6 +164,183 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
     }
 }
 
+// ---------------------------------------------------------------------------
+// Warp-independent combine.  A warp owns one (token, column slice): it classifies
+// the token's picks itself (lanes < k read the routing, then broadcast it with
+// shuffles), so no warp waits at a CTA barrier for another warp's loads.  Lane l
+// takes the row's units l, l + 32, ... of its slice (a unit is VW 32-bit words,
+// 2 * VW bf16 values); PIPE keeps the next unit's k loads in flight while the
+// current unit is reduced.
+// ---------------------------------------------------------------------------
+#ifndef EP_COMBINE_VW
+#define EP_COMBINE_VW 8
+#endif
+#ifndef EP_COMBINE_PIPE
+#define EP_COMBINE_PIPE 1
+#endif
+constexpr int kCombineVW = EP_COMBINE_VW;         // words per unit (4: 16 bytes, 8: 32 bytes)
+constexpr bool kCombinePipe = EP_COMBINE_PIPE != 0;
+constexpr int kCombineWarps = 4;                   // warps per CTA
+
+template <int VW>
+struct VecW {
+    uint32_t w[VW];
+};
+template <int VW>
+__device__ __forceinline__ VecW<VW> ld_vec(const void* p) {
+    VecW<VW> r;
+    if constexpr (VW == 8) {
+        const V8 v = ld_stream_v8(p);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) r.w[e] = v.w[e];
+    } else {
+        const uint4 v = ld_stream_v4(p);
+        r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
+    }
+    return r;
+}
+template <int VW>
+__device__ __forceinline__ void st_vec(void* p, const VecW<VW>& v) {
+    if constexpr (VW == 8) {
+        V8 o;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o.w[e] = v.w[e];
+        st_v8(p, o);
+    } else {
+        st_v4(p, make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
+    }
+}
+
+template <int KM, int VW, bool PIPE>
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_warp_kernel(CombineArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int UB = 4 * VW;  // bytes of a unit
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long item = (long long)blockIdx.x * kCombineWarps + warp;
+    const int t = (int)(item / a.chunks);
+    const int c = (int)(item - (long long)t * a.chunks);
+    const bool live = t < a.B;
+    const bool on = live && !(a.active && !a.active[t]);
+
+    // routing of token t: every lane ends with kind / src / w of each pick
+    const int mine = (live && lane < a.k) ? __ldg(a.topk_idx + (size_t)t * a.k + lane) : -1;
+    int rows[KM];
+    if (a.self_rows) {
+        uint16_t* tab = reinterpret_cast<uint16_t*>(smem + warp * warp_tab_bytes(a.E));
+        zero_warp_tab(tab, a.E);
+        if (live)
+            routing_rows_warp<KM>(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, tab, rows,
+                                  a.expert_offset, a.recv_count);
+        pdl_wait();
+    } else {
+        pdl_wait();
+        const int dp = (live && lane < a.k) ? a.dst_pos[(size_t)t * a.k + lane] : -1;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) rows[j] = __shfl_sync(FULL, dp, j);
+    }
+    pdl_launch_dependents();
+    const float wmine = (live && lane < a.k) ? a.topk_weights[(size_t)t * a.k + lane] : 0.0f;
+    int kind[KM];
+    long long src[KM];
+    float w[KM];
+    unsigned bad = 0;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        const int g = on ? __shfl_sync(FULL, mine, j) : -1;
+        w[j] = __shfl_sync(FULL, wmine, j);
+        kind[j] = kSkip;
+        src[j] = 0;
+        if (j >= a.k || !live) continue;
+        if (g >= 0 && g < a.E) {
+            const int dp = live ? rows[j] : -1;
+            if (dp >= 0 && (long long)dp < a.rows) {
+                kind[j] = kRouted;
+                src[j] = dp;
+            } else if (dp != -1) {
+                bad = EP_ERRBIT_ROW_RANGE;
+            }
+        } else if (g >= a.E + a.Z && g < a.E + a.Z + a.C) {
+            kind[j] = kCopy;
+        } else if (g >= a.E + a.Z + a.C && g < a.E + a.Z + a.C + a.K) {
+            kind[j] = kConst;
+            src[j] = g - (a.E + a.Z + a.C);
+        }
+    }
+    if (lane == 0 && bad) atomicOr(a.err, bad);
+    if (!live) return;
+
+    const int nunits = (a.d * 2) / UB;
+    const char* eo = reinterpret_cast<const char*>(a.expert_out);
+    const char* ox = reinterpret_cast<const char*>(a.ori_x) + (size_t)t * a.d * 2;
+    char* yrow = reinterpret_cast<char*>(a.y) + (size_t)t * a.d * 2;
+    // units of this slice: lane + 32 * (c + chunks * i)
+    auto unit_of = [&](int i) { return lane + 32 * (c + a.chunks * i); };
+    auto issue = [&](VecW<VW> (&buf)[KM], int u) {
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            if (j < a.k && kind[j] == kRouted)
+                buf[j] = ld_vec<VW>(eo + (size_t)src[j] * a.d * 2 + (size_t)u * UB);
+            else if (j < a.k && kind[j] != kSkip)
+                buf[j] = ld_vec<VW>(ox + (size_t)u * UB);
+        }
+    };
+    auto reduce = [&](const VecW<VW> (&buf)[KM], int u) {
+        float acc[2 * VW];
+#pragma unroll
+        for (int e = 0; e < 2 * VW; ++e) acc[e] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            if (j >= a.k || kind[j] == kSkip) continue;
+            float e[2 * VW];
+#pragma unroll
+            for (int q = 0; q < VW; ++q) {
+                e[2 * q] = bf16lo(buf[j].w[q]);
+                e[2 * q + 1] = bf16hi(buf[j].w[q]);
+            }
+            if (kind[j] == kConst) {
+                const size_t off = (size_t)src[j] * a.d * 2 + (size_t)u * UB;
+                const VecW<VW> v1 = ld_vec<VW>(reinterpret_cast<const char*>(a.a1) + off);
+                const VecW<VW> v2 = ld_vec<VW>(reinterpret_cast<const char*>(a.a2) + off);
+                const VecW<VW> vv = ld_vec<VW>(reinterpret_cast<const char*>(a.v) + off);
+#pragma unroll
+                for (int q = 0; q < VW; ++q) {
+                    e[2 * q] = __fadd_rn(__fmul_rn(bf16lo(v1.w[q]), e[2 * q]), __fmul_rn(bf16lo(v2.w[q]), bf16lo(vv.w[q])));
+                    e[2 * q + 1] = __fadd_rn(__fmul_rn(bf16hi(v1.w[q]), e[2 * q + 1]), __fmul_rn(bf16hi(v2.w[q]), bf16hi(vv.w[q])));
+                }
+            }
+#pragma unroll
+            for (int e2 = 0; e2 < 2 * VW; ++e2) acc[e2] = __fmaf_rn(w[j], e[e2], acc[e2]);
+        }
+        VecW<VW> out;
+#pragma unroll
+        for (int q = 0; q < VW; ++q) out.w[q] = pack_bf16x2(acc[2 * q], acc[2 * q + 1]);
+        st_vec<VW>(yrow + (size_t)u * UB, out);
+    };
+
+    if (PIPE) {
+        VecW<VW> cur[KM], nxt[KM];
+        int u = unit_of(0);
+        if (u < nunits) issue(cur, u);
+        for (int i = 0; u < nunits; ++i) {
+            const int un = unit_of(i + 1);
+            if (un < nunits) issue(nxt, un);
+            reduce(cur, u);
+#pragma unroll
+            for (int j = 0; j < KM; ++j) cur[j] = nxt[j];
+            u = un;
+        }
+    } else {
+        for (int i = 0;; ++i) {
+            const int u = unit_of(i);
+            if (u >= nunits) break;
+            VecW<VW> cur[KM];
+            issue(cur, u);
+            reduce(cur, u);
+        }
+    }
+}
+
 }  // namespace
 
 int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
@@ -193,11 +371,43 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
     a.T = s.T;
     a.P = s.P;
     a.M = s.M;
+    a.B = s.B;
     // packed rows also read the layout's counts, complete before the dispatch that
     // precedes this kernel started
     a.self_rows = s.T <= kCombineSelfRowsMaxT ? 1 : 0;
     a.expert_offset = (a.self_rows && s.layout == 1) ? p.expert_offset : nullptr;
     a.recv_count = (a.self_rows && s.layout == 1) ? p.recv_count : nullptr;
+#ifndef EP_COMBINE_OLD
+    {
+        // 32-byte units need every row base it reads or writes 32-byte aligned (rows
+        // are 2d bytes apart, a multiple of 32); otherwise and for k > 8, 16-byte units
+        auto al32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31u) == 0; };
+        const bool wide = kCombineVW == 8 && s.k <= 8 && al32(expert_out) && al32(y) &&
+                          (s.C + s.K == 0 || al32(ori_x)) && (s.K == 0 || (al32(a1) && al32(a2) && al32(v)));
+        const int UB = wide ? 32 : 16;
+        // one warp per (token, column slice): slices only when the batch is too
+        // small to give every SM about eight warps
+        const int nunits = (s.d * 2) / UB;
+        const int max_chunks = (nunits + 31) / 32;
+        long long chunks = (long long)num_sms() * 8 / (s.B > 0 ? s.B : 1);
+        if (chunks < 1) chunks = 1;
+        if (chunks > max_chunks) chunks = max_chunks;
+        a.chunks = (int)chunks;
+        const long long items = (long long)s.B * a.chunks;
+        const long long nblk = (items + kCombineWarps - 1) / kCombineWarps;
+        if (nblk > 0x7fffffffLL) return EP_ERR_UNSUPPORTED;
+        const size_t smem = a.self_rows ? (size_t)kCombineWarps * warp_tab_bytes(s.E) : 0;
+        void (*kern)(CombineArgs);
+        if (s.k <= 4)
+            kern = wide ? combine_warp_kernel<4, 8, kCombinePipe> : combine_warp_kernel<4, 4, kCombinePipe>;
+        else if (s.k <= 8)
+            kern = wide ? combine_warp_kernel<8, 8, kCombinePipe> : combine_warp_kernel<8, 4, kCombinePipe>;
+        else  // 16 picks: 16-byte units without the prefetch, to stay within the registers
+            kern = combine_warp_kernel<16, 4, false>;
+        const cudaError_t e = launch_pdl(kern, dim3((unsigned)nblk), dim3(32 * kCombineWarps), smem, stream, a);
+        return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    }
+#endif
     // One CTA per token when that fills the GPU in about one wave; otherwise split
     // each token's columns over up to nvec / NT CTAs.
     const int nvec = s.d / 8;

@@ -156,6 +156,48 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                  : "memory");
 }
 
+// 32 bytes per thread (sm_100 256-bit global accesses): one load or store moves 16
+// bf16 values, the source of one 16-byte int8 vector.
+struct V8 {
+    uint32_t w[8];
+};
+__device__ __forceinline__ V8 ld_stream_v8(const void* p) {
+    V8 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]),
+                   "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7])
+                 : "l"(p));
+    return r;
+}
+__device__ __forceinline__ void st_v8(void* p, const V8& v) {
+    asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+                 "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+                 "r"(v.w[7])
+                 : "memory");
+}
+
+// 32 bytes at p: one 256-bit access when `wide` (the host has checked that every
+// such address is 32-byte aligned), else two 16-byte accesses (the ABI promises
+// only 16-byte alignment, and an int8 row of d % 32 == 16 bytes leaves every
+// other row on a 16-byte boundary).
+__device__ __forceinline__ V8 ld32(const void* p, bool wide) {
+    if (wide) return ld_stream_v8(p);
+    const uint4 a = ld_stream_v4(p);
+    const uint4 b = ld_stream_v4(reinterpret_cast<const char*>(p) + 16);
+    V8 r;
+    r.w[0] = a.x; r.w[1] = a.y; r.w[2] = a.z; r.w[3] = a.w;
+    r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
+    return r;
+}
+__device__ __forceinline__ void st32(void* p, const V8& v, bool wide) {
+    if (wide) {
+        st_v8(p, v);
+    } else {
+        st_v4(p, make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
+        st_v4(reinterpret_cast<char*>(p) + 16, make_uint4(v.w[4], v.w[5], v.w[6], v.w[7]));
+    }
+}
+
 // bf16 bits <-> fp32: a bf16 is the high half of a binary32.
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -192,6 +234,18 @@ __device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
     const unsigned active = __activemask();
     const unsigned all = __reduce_or_sync(active, bits);
     if (all && (int)(threadIdx.x & 31) == __ffs(active) - 1) atomicOr(err_word, all);
+}
+
+// Shared memory of one warp of the warp-per-token kernels: the routing table
+// (E uint16, 16-byte padded); the dispatch kernels may add a staging row after it.
+__host__ __device__ __forceinline__ int warp_tab_bytes(int E) { return ((2 * E + 15) / 16) * 16; }
+
+// Zero this warp's routing table (E uint16) before its first use.
+__device__ __forceinline__ void zero_warp_tab(uint16_t* tab, int E) {
+    uint32_t* w = reinterpret_cast<uint32_t*>(tab);
+    const int n = warp_tab_bytes(E) / 4;
+    for (int i = threadIdx.x & 31; i < n; i += 32) w[i] = 0u;
+    __syncwarp();
 }
 
 // Receive rows of token t derived from the routing alone, for small per-rank
@@ -256,6 +310,99 @@ __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* acti
         if (g >= 0) row = expert_offset ? s_cnt[threadIdx.x] : g * P * M + r * M + s_cnt[threadIdx.x];
         s_rows[threadIdx.x] = row;
     }
+}
+
+// The same receive rows computed by one warp on its own, for kernels whose warps
+// each own a token (no CTA barrier).  tab: this warp's shared table of E uint16
+// entries, all zero on entry and zero again on return; entry g holds the bit of
+// the pick of this token that routes to g.  An earlier token of the rank looks
+// each of its ids up in the table, so it costs k shared loads instead of k * k
+// compares, and a token counts once per expert however often it repeats an id.
+// On return row[j] is the receive row of pick j (-1: not routed) in every lane.
+template <int KM>
+__device__ __forceinline__ void routing_rows_warp(const int32_t* __restrict__ topk_idx,
+                                                  const uint8_t* active, int t, int k, int E,
+                                                  int T, int P, int M, uint16_t* tab,
+                                                  int (&row)[KM],
+                                                  const int32_t* expert_offset = nullptr,
+                                                  const int32_t* recv_count = nullptr) {
+    static_assert(KM <= 16, "pick bits are kept in 16-bit table entries");
+    const unsigned FULL = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    const bool on = !(active && !active[t]);
+    const int mine = lane < k ? __ldg(topk_idx + (size_t)t * k + lane) : -1;
+    int g[KM];
+    unsigned rb = 0;  // routed picks: an id in [0, E), its first occurrence, token active
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+        g[j] = __shfl_sync(FULL, mine, j);
+        bool routed = on && j < k && g[j] >= 0 && g[j] < E;
+#pragma unroll
+        for (int jj = 0; jj < j; ++jj)
+            if (g[jj] == g[j]) routed = false;
+        if (routed) rb |= 1u << j;
+    }
+    if ((rb >> lane) & 1u) tab[mine] = (uint16_t)(1u << lane);
+    __syncwarp();
+    const int r = t / T;
+    int cnt[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) cnt[j] = 0;
+    const bool vec4 = (k % 4 == 0) && ((reinterpret_cast<uintptr_t>(topk_idx) & 15) == 0);
+    for (int tt = r * T + lane; tt < t; tt += 32) {
+        if (active && !active[tt]) continue;
+        const int32_t* ids = topk_idx + (size_t)tt * k;
+        unsigned hit = 0;
+        if (vec4) {
+#pragma unroll
+            for (int j4 = 0; j4 < KM / 4; ++j4) {
+                if (4 * j4 >= k) continue;
+                const int4 v = __ldg(reinterpret_cast<const int4*>(ids) + j4);
+                hit |= (unsigned)v.x < (unsigned)E ? tab[v.x] : 0u;
+                hit |= (unsigned)v.y < (unsigned)E ? tab[v.y] : 0u;
+                hit |= (unsigned)v.z < (unsigned)E ? tab[v.z] : 0u;
+                hit |= (unsigned)v.w < (unsigned)E ? tab[v.w] : 0u;
+            }
+        } else {
+#pragma unroll
+            for (int jj = 0; jj < KM; ++jj) {
+                if (jj >= k) continue;
+                const int v = __ldg(ids + jj);
+                hit |= (unsigned)v < (unsigned)E ? tab[v] : 0u;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < KM; ++j) cnt[j] += (hit >> j) & 1u;
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j) cnt[j] = (int)__reduce_add_sync(FULL, (unsigned)cnt[j]);
+    if (expert_offset) {
+        // packed: add expert_offset[g] and the r lower ranks' counts of g
+        const int per = r + 1;
+        int part[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j) part[j] = 0;
+        for (int i = lane; i < k * per; i += 32) {
+            const int jsel = i / per, rr = i - jsel * per;
+            int gsel = -1;
+#pragma unroll
+            for (int j = 0; j < KM; ++j)
+                if (j == jsel && ((rb >> j) & 1u)) gsel = g[j];
+            if (gsel < 0) continue;
+            const int val = rr < r ? __ldcg(recv_count + (size_t)gsel * P + rr) : __ldcg(expert_offset + gsel);
+#pragma unroll
+            for (int j = 0; j < KM; ++j)
+                if (j == jsel) part[j] += val;
+        }
+#pragma unroll
+        for (int j = 0; j < KM; ++j) cnt[j] += (int)__reduce_add_sync(FULL, (unsigned)part[j]);
+    }
+    __syncwarp();
+    if ((rb >> lane) & 1u) tab[mine] = 0;
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+        row[j] = ((rb >> j) & 1u) ? (expert_offset ? cnt[j] : g[j] * P * M + r * M + cnt[j]) : -1;
 }
 
 }  // namespace ep
