@@ -220,38 +220,22 @@ def recorded_traffic(workload, kernel):
         return None
 
 
-def oracle_step_sample(w, inp, n_tokens):
-    """One oracle pass (layout, quantize, scatter, combine) over the first
-    n_tokens tokens (a whole number of ranks' worth if possible).  Returns
-    (seconds, algorithmic bytes of that sample)."""
+def oracle_sample_prepare(w, inp, t0, n_tokens):
+    """Inputs of one oracle sample: tokens [t0, t0 + n_tokens) (one logical rank's
+    batch when n_tokens = T) taken as a one-rank problem, plus stand-in expert
+    outputs (the identity expert: dequantized receive rows, made here once and not
+    timed, since the expert computation is not part of dispatch/combine)."""
     import oracle
     from combine_ep_layout_12_b200 import metrics
     B = n_tokens
-    P = max(1, min(w.P, B // max(1, w.T)))
-    if B % P:
-        P = 1
-    M = max(w.M, B // P)
-    cfg = oracle.make_cfg(B, w.d, w.k, P, M, w.E, w.n_zero, w.n_copy, w.n_const, w.quant_mode)
-    idx = np.ascontiguousarray(inp["topk_idx"][:B])
-    x = np.ascontiguousarray(inp["x"][:B])
-    wts = np.ascontiguousarray(inp["topk_weights"][:B])
-    act = None if inp.get("active") is None else np.ascontiguousarray(inp["active"][:B])
-    t0 = time.perf_counter()
-    lay = oracle.layout(cfg, idx, active=act)
-    # scatter into a compact receive buffer (one row per routed pick, same bytes)
-    dp = lay["dst_pos"]
-    compact = np.full(dp.shape, -1, np.int32)
-    routed = dp >= 0
-    n_r = int(routed.sum())
-    compact[routed] = np.arange(n_r, dtype=np.int32)
-    if w.smooth == "expert":
-        rx, rsc = oracle.dispatch_expert_smooth(cfg, x, inp["smooth"], idx, compact, max(n_r, 1))
-    else:
-        q, ts = oracle.quantize(cfg, x, inp["smooth"])
-        rx, rsc = oracle.dispatch(cfg, q, ts, compact, max(n_r, 1))
-    t1 = time.perf_counter()
-    # stand-in expert outputs (bf16 bit patterns) for combine; not part of the
-    # method and not timed
+    cfg = oracle.make_cfg(B, w.d, w.k, 1, B, w.E, w.n_zero, w.n_copy, w.n_const, w.quant_mode)
+    sl = slice(t0, t0 + B)
+    st = {"cfg": cfg, "idx": np.ascontiguousarray(inp["topk_idx"][sl]),
+          "x": np.ascontiguousarray(inp["x"][sl]), "wts": np.ascontiguousarray(inp["topk_weights"][sl]),
+          "act": None if inp.get("active") is None else np.ascontiguousarray(inp["active"][sl]),
+          "smooth": inp["smooth"], "a1": inp["a1"], "a2": inp["a2"], "v": inp["v"],
+          "expert_smooth": w.smooth == "expert", "quant_mode": w.quant_mode, "d": w.d}
+    rx, rsc, compact, n_r = _oracle_dispatch(st)
     if w.quant_mode != 0:
         eo = np.zeros((max(n_r, 1), w.d), np.uint16)
         if n_r:
@@ -261,29 +245,131 @@ def oracle_step_sample(w, inp, n_tokens):
             eo[:n_r] = (f.view(np.uint32) >> 16).astype(np.uint16)
     else:
         eo = rx
-    t2 = time.perf_counter()
-    y = oracle.combine(cfg, eo, idx, wts, compact, x, inp["a1"], inp["a2"], inp["v"], active=act)
-    t3 = time.perf_counter()
-    del y
-    nr, bsp = metrics.routing_counts(w.with_(B=B), idx, n_r, active=act)
-    by = metrics.kernel_bytes(w.with_(B=B, P=P, M=M), nr, bsp, smooth=inp["smooth"] is not None,
-                              masked=act is not None)
-    return (t1 - t0) + (t3 - t2), sum(by.values())
+    st["eo"] = eo
+    nr, bsp = metrics.routing_counts(w.with_(B=B), st["idx"], n_r, active=st["act"])
+    st["bytes"] = sum(metrics.kernel_bytes(w.with_(B=B, P=1, M=B), nr, bsp, smooth=inp["smooth"] is not None,
+                                           masked=st["act"] is not None).values())
+    return st
+
+
+def _oracle_dispatch(st):
+    """Layout, quantization and the scatter into a compact receive buffer (one row
+    per routed pick, the same bytes as the real layout)."""
+    import oracle
+    cfg = st["cfg"]
+    lay = oracle.layout(cfg, st["idx"], active=st["act"])
+    dp = lay["dst_pos"]
+    compact = np.full(dp.shape, -1, np.int32)
+    routed = dp >= 0
+    n_r = int(routed.sum())
+    compact[routed] = np.arange(n_r, dtype=np.int32)
+    if st["expert_smooth"]:
+        rx, rsc = oracle.dispatch_expert_smooth(cfg, st["x"], st["smooth"], st["idx"], compact, max(n_r, 1))
+    else:
+        q, ts = oracle.quantize(cfg, st["x"], st["smooth"])
+        rx, rsc = oracle.dispatch(cfg, q, ts, compact, max(n_r, 1))
+    return rx, rsc, compact, n_r
+
+
+def oracle_sample_run(st):
+    """One timed oracle pass over a prepared sample: layout, quantize, scatter, combine."""
+    import oracle
+    _, _, compact, _ = _oracle_dispatch(st)
+    oracle.combine(st["cfg"], st["eo"], st["idx"], st["wts"], compact, st["x"], st["a1"], st["a2"],
+                   st["v"], active=st["act"])
+
+
+def _oracle_worker_main(conn):
+    """One oracle process: receives its sample once, then runs `reps` passes per
+    request and answers with the seconds they took."""
+    st = conn.recv()
+    while True:
+        msg = conn.recv()
+        if msg[0] != "run":
+            break
+        t = time.perf_counter()
+        for _ in range(msg[1]):
+            oracle_sample_run(st)
+        conn.send(time.perf_counter() - t)
+    conn.close()
+
+
+class OracleWorkers:
+    """One spawned oracle process per host core (at most `cap`), each holding one
+    logical rank's batch of the workload; run(reps) makes every process do reps
+    passes at once and returns each one's seconds."""
+
+    def __init__(self, w, inp, n_tok, cap=32):
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")  # never fork a process that has a CUDA context
+        self.n = max(1, min(os.cpu_count() or 1, cap))
+        n_ranks = max(1, w.B // n_tok)
+        self.states = [oracle_sample_prepare(w, inp, (i % n_ranks) * n_tok, n_tok) for i in range(self.n)]
+        self.conns, self.procs = [], []
+        for st in self.states:
+            a, b = ctx.Pipe()
+            pr = ctx.Process(target=_oracle_worker_main, args=(b,), daemon=True)
+            pr.start()
+            a.send(st)
+            self.conns.append(a)
+            self.procs.append(pr)
+        self.run(1)  # warm: imports and the oracle library loaded in every process
+
+    def run(self, reps):
+        for c in self.conns:
+            c.send(("run", reps))
+        return [c.recv() for c in self.conns]
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send(("stop",))
+            except Exception:
+                pass
+        for pr in self.procs:
+            pr.join(timeout=10)
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def cpu_baseline(w, inp, target_s):
+    """The oracle on the host: single-threaded, then one process per core (up to 32)
+    each running one logical rank's batch, all at once for about target_s seconds.
+    value = algorithmic bytes of all processes' passes / the slowest process's time."""
     n_tok = min(w.B, max(w.T, 1))
-    secs, nbytes, reps = 0.0, 0, 0
-    while secs < target_s or reps < 1:
-        s, b = oracle_step_sample(w, inp, n_tok)
-        secs += s
-        nbytes += b
-        reps += 1
-        if reps >= 1000:
-            break
-    return {"value": nbytes / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": "%d oracle passes over the first %d tokens (one logical rank) of the %s "
-                      "workload, single-threaded C, %.1f s" % (reps, n_tok, w.name, secs)}
+    st = oracle_sample_prepare(w, inp, 0, n_tok)
+    oracle_sample_run(st)
+    t = time.perf_counter()
+    reps1 = 0
+    while time.perf_counter() - t < min(2.0, target_s / 4) or reps1 < 1:
+        oracle_sample_run(st)
+        reps1 += 1
+    t1 = (time.perf_counter() - t) / reps1
+    single = st["bytes"] / t1 / 1e9
+    pool = OracleWorkers(w, inp, n_tok)
+    try:
+        reps = max(1, int(round(target_s / t1)))
+        secs = pool.run(reps)
+    finally:
+        pool.close()
+    nbytes = sum(s["bytes"] for s in pool.states) * reps
+    return {"value": nbytes / max(secs) / 1e9, "unit": "GB/s", "cores": pool.n, "kind": "oracle",
+            "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+            "single_thread_value": single,
+            "sample": "%d oracle processes (spawned, one per host core up to 32), each running %d passes "
+                      "of one logical rank's %d tokens of the %s workload at once; plain C oracle; "
+                      "value = all passes' algorithmic bytes / the slowest process's %.1f s; "
+                      "single_thread_value: one process alone" % (pool.n, reps, n_tok, w.name, max(secs))}
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -297,36 +383,41 @@ def run_reference(args):
     w = wl.get(args.workload)
     inp = wl.generate(w)
     n_tok = min(w.B, max(w.T, 1))
-    for _ in range(args.warmup):
-        oracle_step_sample(w, inp, n_tok)
-    secs, nbytes = 0.0, 0
-    for _ in range(args.steps):
-        s, b = oracle_step_sample(w, inp, n_tok)
-        secs += s
-        nbytes += b
-    value = nbytes / secs / 1e9
-    sample = "%d oracle passes over the first %d tokens (one logical rank) of the %s workload, " \
-             "single-threaded C" % (args.steps, n_tok, w.name)
+    pool = OracleWorkers(w, inp, n_tok)
+    try:
+        for _ in range(args.warmup):
+            pool.run(1)
+        total = 0.0
+        for _ in range(args.steps):  # a step: every process does one pass at once
+            total += max(pool.run(1))
+    finally:
+        pool.close()
+    nbytes = sum(s["bytes"] for s in pool.states) * args.steps
+    value = nbytes / total / 1e9
+    sample = ("%d oracle processes (spawned, one per host core up to 32), each doing one pass of one "
+              "logical rank's %d tokens of the %s workload per step; plain C oracle; step time = the "
+              "slowest process's pass" % (pool.n, n_tok, w.name))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": config_dict(w, args),
-        "tokens_per_s": n_tok * args.steps / secs,
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "data": "synthetic", "config": config_dict(w),
+        "tokens_per_s": pool.n * n_tok * args.steps / total,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": pool.n, "kind": "oracle",
+                         "cpu_model": cpu_model(), "host_cpus": os.cpu_count(), "sample": sample},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def config_dict(w, args):
+def config_dict(w):
+    """The workload only (both arms report the same dict); how it was timed goes
+    under the line's "method" key."""
     return {"workload": w.name, "B": w.B, "d": w.d, "E": w.E, "k": w.k, "P": w.P, "M": w.M,
             "n_zero": w.n_zero, "n_copy": w.n_copy, "n_const": w.n_const,
             "quant_mode": w.quant_mode, "payload": "int8" if w.quant_mode != 0 else "bf16",
-            "routing": w.routing, "layout": "low-latency [E, P*M, d]",
-            "l2": ("flushed between steps (%d MB memset, outside the step events)" % args.flush_mb)
-            if args.flush_mb else "not flushed",
+            "routing": w.routing, "layout": "packed [B*k, d]" if w.layout == 1 else "low-latency [E, P*M, d]",
             "parallelism": "replicas (logical EP ranks inside each GPU)"}
 
 
@@ -683,19 +774,22 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    cfg = config_dict(w, args)
-    if R > 1:
-        cfg["l2"] = ("%d buffer sets in rotation: consecutive steps touch disjoint memory "
-                     "(%.0f MB algorithmic per step, L2 126 MB)" % (R, wb.step_bytes / 1e6))
-    cfg["timing"] = ("K steps as replays of a CUDA graph of %d consecutive steps (ep_layout_dispatch -> "
-                     "ep_combine, programmatic launch edges), CUDA events around the whole timed region; "
-                     "step_latency_us_median: single-step graph replays with events around each" % S)
+    cfg = config_dict(w)
+    method = {
+        "l2": ("%d buffer sets in rotation: consecutive steps touch disjoint memory "
+               "(%.0f MB algorithmic per step, L2 126 MB)" % (R, wb.step_bytes / 1e6)) if R > 1 else
+              ("flushed between steps (%d MB memset, timed alone and subtracted)" % args.flush_mb),
+        "timing": ("K steps as replays of a CUDA graph of %d consecutive steps (ep_layout_dispatch -> "
+                   "ep_combine, programmatic launch edges), CUDA events around the whole timed region; "
+                   "step_latency_us_median: single-step graph replays with events around each" % S),
+    }
     lps = wb.launches_per_step
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": 1e3 * job_s / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": cfg,
+        "method": method,
         "tokens_per_s": job_tokens / job_s,
         "bytes_per_step": wb.step_bytes,
         "step_latency_us_median": 1e3 * statistics.median(step_ms),

@@ -37,6 +37,32 @@ class ep_buffer_ptrs(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in BUFFER_FIELDS]
 
 
+SHARD_MAX_RANKS = 64
+
+
+class ep_shard_table(ctypes.Structure):
+    _fields_ = [("rank", ctypes.c_int32),
+                ("recv_x", ctypes.c_void_p * SHARD_MAX_RANKS),
+                ("recv_scale", ctypes.c_void_p * SHARD_MAX_RANKS),
+                ("recv_src", ctypes.c_void_p * SHARD_MAX_RANKS)]
+
+
+def make_shard_table(rank, recv_x, recv_scale=None, recv_src=None):
+    """ep_shard_table from per-rank device addresses (lists of ints; None entries or
+    lists mean NULL)."""
+    t = ep_shard_table()
+    t.rank = int(rank)
+    for name, vals in (("recv_x", recv_x), ("recv_scale", recv_scale), ("recv_src", recv_src)):
+        if vals is None:
+            continue
+        if len(vals) > SHARD_MAX_RANKS:
+            raise ValueError("at most %d ranks" % SHARD_MAX_RANKS)
+        arr = getattr(t, name)
+        for q, v in enumerate(vals):
+            arr[q] = v
+    return t
+
+
 class EPError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
@@ -85,9 +111,15 @@ def _load(path):
     L.ep_combine.argtypes = [vp] * 11
     L.ep_buffer_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     L.ep_layout_static_scratch.argtypes = [ctypes.POINTER(ep_config)] + [vp] * 8
+    L.ep_shard_workspace_size.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ctypes.c_size_t)]
+    L.ep_shard_layout.argtypes = [ctypes.POINTER(ep_config), ctypes.c_int32] + [vp] * 6
+    L.ep_shard_dispatch.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 6
+    L.ep_shard_combine.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 11
+    L.ep_shard_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     for f in (L.ep_buffer_size, L.ep_buffer_create, L.ep_buffer_destroy, L.ep_layout,
               L.ep_dispatch, L.ep_layout_dispatch, L.ep_combine, L.ep_buffer_check,
-              L.ep_layout_static_scratch):
+              L.ep_layout_static_scratch, L.ep_shard_workspace_size, L.ep_shard_layout,
+              L.ep_shard_dispatch, L.ep_shard_combine, L.ep_shard_check):
         f.restype = i
     L.ep_status_str.argtypes = [i]
     L.ep_status_str.restype = ctypes.c_char_p
@@ -158,3 +190,32 @@ def ep_layout_static_scratch(cfg, topk_idx, expert_count, expert_offset, recv_co
     _check(lib().ep_layout_static_scratch(ctypes.byref(cfg), topk_idx, expert_count,
                                           expert_offset, recv_count, dst_pos, recv_src,
                                           err_word, stream), "ep_layout_static_scratch")
+
+
+def ep_shard_workspace_size(cfg):
+    n = ctypes.c_size_t()
+    _check(lib().ep_shard_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "ep_shard_workspace_size")
+    return int(n.value)
+
+
+def ep_shard_layout(cfg, rank, topk_idx, x_active_mask, dst_pos, send_count, workspace, stream=0):
+    _check(lib().ep_shard_layout(ctypes.byref(cfg), int(rank), topk_idx, x_active_mask, dst_pos,
+                                 send_count, workspace, stream), "ep_shard_layout")
+
+
+def ep_shard_dispatch(cfg, table, x, smooth_scale, dst_pos, token_scale, workspace, stream=0):
+    _check(lib().ep_shard_dispatch(ctypes.byref(cfg), ctypes.byref(table), x, smooth_scale, dst_pos,
+                                   token_scale, workspace, stream), "ep_shard_dispatch")
+
+
+def ep_shard_combine(cfg, table, topk_idx, topk_weights, x_active_mask, dst_pos, ori_x, a1, a2, v, y,
+                     workspace, stream=0):
+    _check(lib().ep_shard_combine(ctypes.byref(cfg), ctypes.byref(table), topk_idx, topk_weights,
+                                  x_active_mask, dst_pos, ori_x, a1, a2, v, y, workspace, stream),
+           "ep_shard_combine")
+
+
+def ep_shard_check(workspace, stream=0):
+    bits = ctypes.c_uint32()
+    _check(lib().ep_shard_check(workspace, stream, ctypes.byref(bits)), "ep_shard_check")
+    return int(bits.value)

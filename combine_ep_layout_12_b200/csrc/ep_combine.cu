@@ -22,7 +22,11 @@
 namespace ep {
 namespace {
 
-enum : int { kSkip = 0, kRouted = 1, kCopy = 2, kConst = 3 };
+#ifndef EP_COMBINE_PREFETCH
+#define EP_COMBINE_PREFETCH 0
+#endif
+// Column blocks (one per CTA pass over the row) prefetched into L2 ahead of the loads.
+constexpr int kCombinePrefetch = EP_COMBINE_PREFETCH;
 
 // Per-rank batches up to this size derive their rows from the routing (the scan of
 // the earlier tokens' ids stays within one load per thread).  At 256 tokens per
@@ -49,7 +53,6 @@ struct CombineArgs {
     const int32_t* expert_offset;  // packed rows with self_rows: the layout's counts
     const int32_t* recv_count;
     int T, P, M;
-    int B;                       // tokens
 };
 
 __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
@@ -61,11 +64,27 @@ __device__ __forceinline__ void unpack8(const uint4& r, float* f) {
     }
 }
 
-template <int KMAX>
-__global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(CombineArgs a) {
-    __shared__ int s_kind[KMAX];
-    __shared__ long long s_src[KMAX];  // receive row (routed) or const index
+// Where the expert output of a routed row lives: this buffer's expert_out, or the
+// slab of the rank that owns the row's expert (see ShardTable).
+struct LocalOut {
+    __device__ __forceinline__ const uint16_t* row(const CombineArgs& a, int r) const {
+        return a.expert_out + (size_t)r * a.d;
+    }
+};
+struct ShardOut {
+    const ShardTable& tab;
+    __device__ __forceinline__ const uint16_t* row(const CombineArgs& a, int r) const {
+        const int q = (int)(r / tab.slab_rows);
+        return reinterpret_cast<const uint16_t*>(tab.x[q]) + (size_t)(r - q * tab.slab_rows) * a.d;
+    }
+};
+
+template <int KMAX, class Out>
+__device__ __forceinline__ void combine_body(const CombineArgs& a, const Out& out_rows) {
+    __shared__ const uint16_t* s_ptr[KMAX];  // row the pick reads (expert output or ori_x[t]); null: no term
     __shared__ float s_w[KMAX];
+    __shared__ int s_const[KMAX];            // constant expert index, -1 for other picks
+    __shared__ uint16_t s_tab[kMaxE];
 
     // CTA = (token t, column slice c); the slice is swept by the CTA's threads
     const int t = blockIdx.x / a.chunks;
@@ -80,8 +99,11 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
     // griddepcontrol.wait and overlaps their tail; the expert outputs are read and
     // y is written only after the wait.
     __shared__ int s_rows[KMAX], s_g[KMAX], s_cnt[KMAX];
+    // the weights were final before the preceding kernels started (as topk_idx):
+    // their load is issued first so its latency overlaps the row lookup
+    const float wt = threadIdx.x < a.k ? a.topk_weights[(size_t)t * a.k + threadIdx.x] : 0.0f;
     if (a.self_rows) {
-        routing_rows(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt,
+        routing_rows(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt, s_tab,
                      a.expert_offset, a.recv_count);
     } else {
         pdl_wait();
@@ -89,60 +111,71 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
     pdl_launch_dependents();
 
     unsigned bad = 0;
+    int is_const = 0;
     const bool on = !(a.active && !a.active[t]);  // an inactive token has no terms
     if (threadIdx.x < a.k) {
         const size_t i = (size_t)t * a.k + threadIdx.x;
         const int g = on ? a.topk_idx[i] : -1;
         const int dp = a.self_rows ? s_rows[threadIdx.x] : a.dst_pos[i];
-        int kind = kSkip;
-        long long src = 0;
+        const uint16_t* ptr = nullptr;
+        int cidx = -1;
         if (g >= 0 && g < a.E) {
-            if (dp >= 0 && (long long)dp < a.rows) {
-                kind = kRouted;
-                src = dp;
-            } else if (dp != -1) {
+            if (dp >= 0 && (long long)dp < a.rows)
+                ptr = out_rows.row(a, dp);
+            else if (dp != -1)
                 bad = EP_ERRBIT_ROW_RANGE;
-            }
         } else if (g >= a.E + a.Z && g < a.E + a.Z + a.C) {
-            kind = kCopy;
+            ptr = a.ori_x + (size_t)t * a.d;  // copy expert
         } else if (g >= a.E + a.Z + a.C && g < a.E + a.Z + a.C + a.K) {
-            kind = kConst;
-            src = g - (a.E + a.Z + a.C);
+            ptr = a.ori_x + (size_t)t * a.d;  // constant expert: a1[c] * ori_x + a2[c] * v[c]
+            cidx = g - (a.E + a.Z + a.C);
+            is_const = 1;
         }
-        s_kind[threadIdx.x] = kind;
-        s_src[threadIdx.x] = src;
-        s_w[threadIdx.x] = a.topk_weights[i];
+        s_ptr[threadIdx.x] = ptr;
+        s_w[threadIdx.x] = wt;
+        s_const[threadIdx.x] = cidx;
     }
     if (a.self_rows) pdl_wait();
     if (threadIdx.x < 32) report_err(a.err, bad);
-    __syncthreads();
+    const int any_const = __syncthreads_or(is_const);
 
-    for (int vcol = v_begin + threadIdx.x; vcol < v_end; vcol += blockDim.x) {
+    // picks with a term (CTA-uniform): skipped picks add nothing, exactly as if absent
+    unsigned live = 0;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+        if (j < a.k && s_ptr[j] != nullptr) live |= 1u << j;
+
+    // L2 prefetch, kCombinePrefetch column blocks ahead of the CTA's loads: thread j
+    // asks the copy engine for pick j's next block of row bytes, so more of the
+    // row is in flight than the loads' registers hold
+    const int NT = blockDim.x;
+    auto prefetch = [&](int blk) {
+        const int j = threadIdx.x;
+        const int v0 = v_begin + blk * NT;
+        if (kCombinePrefetch > 0 && j < KMAX && ((live >> j) & 1u) && v0 < v_end) {
+            const int nv = min(NT, v_end - v0);
+            bulk_prefetch_l2(s_ptr[j] + (size_t)v0 * 8, (uint32_t)nv * 16u);
+        }
+    };
+    for (int b = 0; b < kCombinePrefetch; ++b) prefetch(b);
+    int blk = 0;
+    for (int vcol = v_begin + threadIdx.x; vcol < v_end; vcol += blockDim.x, ++blk) {
+        if (kCombinePrefetch > 0) prefetch(blk + kCombinePrefetch);
         const size_t col = (size_t)vcol * 8;
         uint4 raw[KMAX];
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            raw[j] = make_uint4(0, 0, 0, 0);
-            if (j < a.k) {
-                const int kind = s_kind[j];
-                if (kind == kRouted)
-                    raw[j] = ld_stream_v4(a.expert_out + (size_t)s_src[j] * a.d + col);
-                else if (kind != kSkip)
-                    raw[j] = ld_stream_v4(a.ori_x + (size_t)t * a.d + col);
-            }
-        }
+        for (int j = 0; j < KMAX; ++j)
+            raw[j] = ((live >> j) & 1u) ? ld_stream_v4(s_ptr[j] + col) : make_uint4(0, 0, 0, 0);
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
 #pragma unroll
         for (int j = 0; j < KMAX; ++j) {
-            if (j >= a.k) continue;
-            const int kind = s_kind[j];
-            if (kind == kSkip) continue;
+            if (!((live >> j) & 1u)) continue;
             float e[8];
             unpack8(raw[j], e);
-            if (kind == kConst) {
-                const size_t off = (size_t)s_src[j] * a.d + col;
+            if (any_const && s_const[j] >= 0) {
+                const size_t off = (size_t)s_const[j] * a.d + col;
                 float f1[8], f2[8], fv[8];
                 unpack8(ld_stream_v4(a.a1 + off), f1);
                 unpack8(ld_stream_v4(a.a2 + off), f2);
@@ -164,190 +197,25 @@ __global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(Combin
     }
 }
 
-// ---------------------------------------------------------------------------
-// Warp-independent combine.  A warp owns one (token, column slice): it classifies
-// the token's picks itself (lanes < k read the routing, then broadcast it with
-// shuffles), so no warp waits at a CTA barrier for another warp's loads.  Lane l
-// takes the row's units l, l + 32, ... of its slice (a unit is VW 32-bit words,
-// 2 * VW bf16 values); PIPE keeps the next unit's k loads in flight while the
-// current unit is reduced.
-// ---------------------------------------------------------------------------
-#ifndef EP_COMBINE_VW
-#define EP_COMBINE_VW 8
-#endif
-#ifndef EP_COMBINE_PIPE
-#define EP_COMBINE_PIPE 1
-#endif
-constexpr int kCombineVW = EP_COMBINE_VW;         // words per unit (4: 16 bytes, 8: 32 bytes)
-constexpr bool kCombinePipe = EP_COMBINE_PIPE != 0;
-constexpr int kCombineWarps = 4;                   // warps per CTA
-
-template <int VW>
-struct VecW {
-    uint32_t w[VW];
-};
-template <int VW>
-__device__ __forceinline__ VecW<VW> ld_vec(const void* p) {
-    VecW<VW> r;
-    if constexpr (VW == 8) {
-        const V8 v = ld_stream_v8(p);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) r.w[e] = v.w[e];
-    } else {
-        const uint4 v = ld_stream_v4(p);
-        r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
-    }
-    return r;
-}
-template <int VW>
-__device__ __forceinline__ void st_vec(void* p, const VecW<VW>& v) {
-    if constexpr (VW == 8) {
-        V8 o;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o.w[e] = v.w[e];
-        st_v8(p, o);
-    } else {
-        st_v4(p, make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
-    }
+template <int KMAX>
+__global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8)) combine_kernel(CombineArgs a) {
+    combine_body<KMAX>(a, LocalOut());
 }
 
-template <int KM, int VW, bool PIPE>
-__global__ void __launch_bounds__(32 * kCombineWarps) combine_warp_kernel(CombineArgs a) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    constexpr unsigned FULL = 0xffffffffu;
-    constexpr int UB = 4 * VW;  // bytes of a unit
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const long long item = (long long)blockIdx.x * kCombineWarps + warp;
-    const int t = (int)(item / a.chunks);
-    const int c = (int)(item - (long long)t * a.chunks);
-    const bool live = t < a.B;
-    const bool on = live && !(a.active && !a.active[t]);
-
-    // routing of token t: every lane ends with kind / src / w of each pick
-    const int mine = (live && lane < a.k) ? __ldg(a.topk_idx + (size_t)t * a.k + lane) : -1;
-    int rows[KM];
-    if (a.self_rows) {
-        uint16_t* tab = reinterpret_cast<uint16_t*>(smem + warp * warp_tab_bytes(a.E));
-        zero_warp_tab(tab, a.E);
-        if (live)
-            routing_rows_warp<KM>(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, tab, rows,
-                                  a.expert_offset, a.recv_count);
-        pdl_wait();
-    } else {
-        pdl_wait();
-        const int dp = (live && lane < a.k) ? a.dst_pos[(size_t)t * a.k + lane] : -1;
-#pragma unroll
-        for (int j = 0; j < KM; ++j) rows[j] = __shfl_sync(FULL, dp, j);
-    }
-    pdl_launch_dependents();
-    const float wmine = (live && lane < a.k) ? a.topk_weights[(size_t)t * a.k + lane] : 0.0f;
-    int kind[KM];
-    long long src[KM];
-    float w[KM];
-    unsigned bad = 0;
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        const int g = on ? __shfl_sync(FULL, mine, j) : -1;
-        w[j] = __shfl_sync(FULL, wmine, j);
-        kind[j] = kSkip;
-        src[j] = 0;
-        if (j >= a.k || !live) continue;
-        if (g >= 0 && g < a.E) {
-            const int dp = live ? rows[j] : -1;
-            if (dp >= 0 && (long long)dp < a.rows) {
-                kind[j] = kRouted;
-                src[j] = dp;
-            } else if (dp != -1) {
-                bad = EP_ERRBIT_ROW_RANGE;
-            }
-        } else if (g >= a.E + a.Z && g < a.E + a.Z + a.C) {
-            kind[j] = kCopy;
-        } else if (g >= a.E + a.Z + a.C && g < a.E + a.Z + a.C + a.K) {
-            kind[j] = kConst;
-            src[j] = g - (a.E + a.Z + a.C);
-        }
-    }
-    if (lane == 0 && bad) atomicOr(a.err, bad);
-    if (!live) return;
-
-    const int nunits = (a.d * 2) / UB;
-    const char* eo = reinterpret_cast<const char*>(a.expert_out);
-    const char* ox = reinterpret_cast<const char*>(a.ori_x) + (size_t)t * a.d * 2;
-    char* yrow = reinterpret_cast<char*>(a.y) + (size_t)t * a.d * 2;
-    // units of this slice: lane + 32 * (c + chunks * i)
-    auto unit_of = [&](int i) { return lane + 32 * (c + a.chunks * i); };
-    auto issue = [&](VecW<VW> (&buf)[KM], int u) {
-#pragma unroll
-        for (int j = 0; j < KM; ++j) {
-            if (j < a.k && kind[j] == kRouted)
-                buf[j] = ld_vec<VW>(eo + (size_t)src[j] * a.d * 2 + (size_t)u * UB);
-            else if (j < a.k && kind[j] != kSkip)
-                buf[j] = ld_vec<VW>(ox + (size_t)u * UB);
-        }
-    };
-    auto reduce = [&](const VecW<VW> (&buf)[KM], int u) {
-        float acc[2 * VW];
-#pragma unroll
-        for (int e = 0; e < 2 * VW; ++e) acc[e] = 0.0f;
-#pragma unroll
-        for (int j = 0; j < KM; ++j) {
-            if (j >= a.k || kind[j] == kSkip) continue;
-            float e[2 * VW];
-#pragma unroll
-            for (int q = 0; q < VW; ++q) {
-                e[2 * q] = bf16lo(buf[j].w[q]);
-                e[2 * q + 1] = bf16hi(buf[j].w[q]);
-            }
-            if (kind[j] == kConst) {
-                const size_t off = (size_t)src[j] * a.d * 2 + (size_t)u * UB;
-                const VecW<VW> v1 = ld_vec<VW>(reinterpret_cast<const char*>(a.a1) + off);
-                const VecW<VW> v2 = ld_vec<VW>(reinterpret_cast<const char*>(a.a2) + off);
-                const VecW<VW> vv = ld_vec<VW>(reinterpret_cast<const char*>(a.v) + off);
-#pragma unroll
-                for (int q = 0; q < VW; ++q) {
-                    e[2 * q] = __fadd_rn(__fmul_rn(bf16lo(v1.w[q]), e[2 * q]), __fmul_rn(bf16lo(v2.w[q]), bf16lo(vv.w[q])));
-                    e[2 * q + 1] = __fadd_rn(__fmul_rn(bf16hi(v1.w[q]), e[2 * q + 1]), __fmul_rn(bf16hi(v2.w[q]), bf16hi(vv.w[q])));
-                }
-            }
-#pragma unroll
-            for (int e2 = 0; e2 < 2 * VW; ++e2) acc[e2] = __fmaf_rn(w[j], e[e2], acc[e2]);
-        }
-        VecW<VW> out;
-#pragma unroll
-        for (int q = 0; q < VW; ++q) out.w[q] = pack_bf16x2(acc[2 * q], acc[2 * q + 1]);
-        st_vec<VW>(yrow + (size_t)u * UB, out);
-    };
-
-    if (PIPE) {
-        VecW<VW> cur[KM], nxt[KM];
-        int u = unit_of(0);
-        if (u < nunits) issue(cur, u);
-        for (int i = 0; u < nunits; ++i) {
-            const int un = unit_of(i + 1);
-            if (un < nunits) issue(nxt, un);
-            reduce(cur, u);
-#pragma unroll
-            for (int j = 0; j < KM; ++j) cur[j] = nxt[j];
-            u = un;
-        }
-    } else {
-        for (int i = 0;; ++i) {
-            const int u = unit_of(i);
-            if (u >= nunits) break;
-            VecW<VW> cur[KM];
-            issue(cur, u);
-            reduce(cur, u);
-        }
-    }
+// Multi-GPU form: expert outputs read from every rank's slab (peer loads).
+template <int KMAX>
+__global__ void __launch_bounds__(128, (KMAX > 8 ? 4 : 8))
+    combine_shard_kernel(CombineArgs a, const __grid_constant__ ShardTable tab) {
+    combine_body<KMAX>(a, ShardOut{tab});
 }
 
 }  // namespace
 
-int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
-                   const int32_t* topk_idx, const float* topk_weights, const uint8_t* active,
-                   const uint16_t* ori_x,
-                   const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
-                   cudaStream_t stream) {
+namespace {
+int launch_combine_impl(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
+                        const int32_t* topk_idx, const float* topk_weights, const uint8_t* active,
+                        const uint16_t* ori_x, const uint16_t* a1, const uint16_t* a2,
+                        const uint16_t* v, uint16_t* y, cudaStream_t stream, const ShardTable* tab) {
     if (s.B == 0) return EP_OK;
     CombineArgs a;
     a.expert_out = expert_out;
@@ -371,43 +239,11 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
     a.T = s.T;
     a.P = s.P;
     a.M = s.M;
-    a.B = s.B;
     // packed rows also read the layout's counts, complete before the dispatch that
     // precedes this kernel started
-    a.self_rows = s.T <= kCombineSelfRowsMaxT ? 1 : 0;
+    a.self_rows = (tab == nullptr && s.T <= kCombineSelfRowsMaxT) ? 1 : 0;
     a.expert_offset = (a.self_rows && s.layout == 1) ? p.expert_offset : nullptr;
     a.recv_count = (a.self_rows && s.layout == 1) ? p.recv_count : nullptr;
-#ifndef EP_COMBINE_OLD
-    {
-        // 32-byte units need every row base it reads or writes 32-byte aligned (rows
-        // are 2d bytes apart, a multiple of 32); otherwise and for k > 8, 16-byte units
-        auto al32 = [](const void* q) { return (reinterpret_cast<uintptr_t>(q) & 31u) == 0; };
-        const bool wide = kCombineVW == 8 && s.k <= 8 && al32(expert_out) && al32(y) &&
-                          (s.C + s.K == 0 || al32(ori_x)) && (s.K == 0 || (al32(a1) && al32(a2) && al32(v)));
-        const int UB = wide ? 32 : 16;
-        // one warp per (token, column slice): slices only when the batch is too
-        // small to give every SM about eight warps
-        const int nunits = (s.d * 2) / UB;
-        const int max_chunks = (nunits + 31) / 32;
-        long long chunks = (long long)num_sms() * 8 / (s.B > 0 ? s.B : 1);
-        if (chunks < 1) chunks = 1;
-        if (chunks > max_chunks) chunks = max_chunks;
-        a.chunks = (int)chunks;
-        const long long items = (long long)s.B * a.chunks;
-        const long long nblk = (items + kCombineWarps - 1) / kCombineWarps;
-        if (nblk > 0x7fffffffLL) return EP_ERR_UNSUPPORTED;
-        const size_t smem = a.self_rows ? (size_t)kCombineWarps * warp_tab_bytes(s.E) : 0;
-        void (*kern)(CombineArgs);
-        if (s.k <= 4)
-            kern = wide ? combine_warp_kernel<4, 8, kCombinePipe> : combine_warp_kernel<4, 4, kCombinePipe>;
-        else if (s.k <= 8)
-            kern = wide ? combine_warp_kernel<8, 8, kCombinePipe> : combine_warp_kernel<8, 4, kCombinePipe>;
-        else  // 16 picks: 16-byte units without the prefetch, to stay within the registers
-            kern = combine_warp_kernel<16, 4, false>;
-        const cudaError_t e = launch_pdl(kern, dim3((unsigned)nblk), dim3(32 * kCombineWarps), smem, stream, a);
-        return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
-    }
-#endif
     // One CTA per token when that fills the GPU in about one wave; otherwise split
     // each token's columns over up to nvec / NT CTAs.
     const int nvec = s.d / 8;
@@ -422,7 +258,16 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
     if (nblocks > 0x7fffffffLL) return EP_ERR_UNSUPPORTED;
     const dim3 grid((unsigned)nblocks);
     cudaError_t e;
-    if (s.k <= 2)
+    if (tab) {
+        if (s.k <= 2)
+            e = launch_pdl(combine_shard_kernel<2>, grid, dim3(NT), 0, stream, a, *tab);
+        else if (s.k <= 4)
+            e = launch_pdl(combine_shard_kernel<4>, grid, dim3(NT), 0, stream, a, *tab);
+        else if (s.k <= 8)
+            e = launch_pdl(combine_shard_kernel<8>, grid, dim3(NT), 0, stream, a, *tab);
+        else
+            e = launch_pdl(combine_shard_kernel<16>, grid, dim3(NT), 0, stream, a, *tab);
+    } else if (s.k <= 2)
         e = launch_pdl(combine_kernel<2>, grid, dim3(NT), 0, stream, a);
     else if (s.k <= 4)
         e = launch_pdl(combine_kernel<4>, grid, dim3(NT), 0, stream, a);
@@ -431,6 +276,24 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
     else
         e = launch_pdl(combine_kernel<16>, grid, dim3(NT), 0, stream, a);
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+}  // namespace
+
+int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expert_out,
+                   const int32_t* topk_idx, const float* topk_weights, const uint8_t* active,
+                   const uint16_t* ori_x,
+                   const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
+                   cudaStream_t stream) {
+    return launch_combine_impl(s, p, expert_out, topk_idx, topk_weights, active, ori_x, a1, a2, v, y,
+                               stream, nullptr);
+}
+
+int launch_shard_combine(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
+                         const float* topk_weights, const uint8_t* active, const uint16_t* ori_x,
+                         const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
+                         const ShardTable& tab, cudaStream_t stream) {
+    return launch_combine_impl(s, p, nullptr, topk_idx, topk_weights, active, ori_x, a1, a2, v, y,
+                               stream, &tab);
 }
 
 }  // namespace ep

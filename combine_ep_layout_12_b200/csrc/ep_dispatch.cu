@@ -43,54 +43,21 @@ __global__ void __launch_bounds__(256) dispatch_bf16_kernel(DispatchArgs a) {
     if (a.self_rows) pdl_wait();
 }
 
-// Warp-per-token dispatch (rows up to 8192 elements): kWarpTokens tokens per CTA,
-// one per warp.  Same PDL placement as the kernels above.
-template <int NU, int MODE, int KM, bool BULK>
-__global__ void __launch_bounds__(32 * kWarpTokens) dispatch_warp_kernel(DispatchArgs a) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    if (!a.self_rows) pdl_wait();
+// Multi-GPU form: rows read from dst_pos, stored into the owning rank's slab.
+template <int U, bool STATIC>
+__global__ void __launch_bounds__(256)
+    dispatch_int8_shard_kernel(DispatchArgs a, const __grid_constant__ ShardTable tab) {
+    pdl_wait();
     pdl_launch_dependents();
-    const int warp = threadIdx.x >> 5;
-    const int t = blockIdx.x * kWarpTokens + warp;
-    const size_t per = (size_t)warp_tab_bytes(a.E) + (BULK ? (size_t)a.d : 0);
-    unsigned char* mine = smem + warp * per;
-    uint16_t* tab = reinterpret_cast<uint16_t*>(mine);
-    if (t < a.B) {
-        if (a.self_rows) zero_warp_tab(tab, a.E);
-        dispatch_warp_body<NU, MODE, KM, BULK>(a, t, tab, mine + warp_tab_bytes(a.E));
-    }
-    if (a.self_rows) pdl_wait();
+    dispatch_int8_body<U, STATIC>(a, blockIdx.x, ShardRows{tab});
 }
 
-using DispatchKernel = void (*)(DispatchArgs);
-
-template <int MODE, int KM>
-DispatchKernel warp_kernel_nu(int NU) {
-    constexpr bool BULK = MODE != 0 && kDispatchBulk;
-    if constexpr (MODE == 0) {
-        switch (NU) {
-            case 2: return dispatch_warp_kernel<2, MODE, KM, BULK>;
-            case 4: return dispatch_warp_kernel<4, MODE, KM, BULK>;
-            case 8: return dispatch_warp_kernel<8, MODE, KM, BULK>;
-            case 14: return dispatch_warp_kernel<14, MODE, KM, BULK>;
-            default: return dispatch_warp_kernel<16, MODE, KM, BULK>;
-        }
-    } else {
-        switch (NU) {
-            case 1: return dispatch_warp_kernel<1, MODE, KM, BULK>;
-            case 2: return dispatch_warp_kernel<2, MODE, KM, BULK>;
-            case 4: return dispatch_warp_kernel<4, MODE, KM, BULK>;
-            case 7: return dispatch_warp_kernel<7, MODE, KM, BULK>;
-            default: return dispatch_warp_kernel<8, MODE, KM, BULK>;
-        }
-    }
-}
-
-// The warp-per-token kernel for quant_mode `mode`, k picks and NU units per lane.
-DispatchKernel pick_warp_kernel(int mode, int k, int NU) {
-    if (mode == 0) return k <= 8 ? warp_kernel_nu<0, 8>(NU) : warp_kernel_nu<0, 16>(NU);
-    if (mode == 1) return k <= 8 ? warp_kernel_nu<1, 8>(NU) : warp_kernel_nu<1, 16>(NU);
-    return k <= 8 ? warp_kernel_nu<2, 8>(NU) : warp_kernel_nu<2, 16>(NU);
+template <int U>
+__global__ void __launch_bounds__(256)
+    dispatch_bf16_shard_kernel(DispatchArgs a, const __grid_constant__ ShardTable tab) {
+    pdl_wait();
+    pdl_launch_dependents();
+    dispatch_bf16_body<U>(a, blockIdx.x, ShardRows{tab});
 }
 
 template <bool STATIC>
@@ -385,19 +352,6 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
     cudaError_t e = cudaSuccess;
     const dim3 grid(s.B);
     if (a.expert_smooth) return launch_dispatch_expert(s, p, x, smooth, stream);
-    const int NU = warp_units(s.quant_mode, s.d);
-    if (NU > 0) {
-        const size_t smem = dispatch_warp_smem(s.E, s.d, s.quant_mode != 0 && kDispatchBulk, kWarpTokens);
-        const DispatchKernel kern = pick_warp_kernel(s.quant_mode, s.k, NU);
-        // above the default 48 KB (E up to 2048, staging rows up to 8 KB) the kernel
-        // needs the opt-in; setting it is idempotent
-        if (smem > 48 * 1024 &&
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return EP_ERR_CUDA;
-        const dim3 wgrid((unsigned)((s.B + kWarpTokens - 1) / kWarpTokens));
-        e = launch_pdl(kern, wgrid, dim3(32 * kWarpTokens), smem, stream, a);
-        return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
-    }
     if (s.quant_mode != 0) {
         if (pick_units(s.d / 16, 8, &U, &NT) != EP_OK) return EP_ERR_UNSUPPORTED;
         e = s.quant_mode == 1 ? launch_int8<true>(U, grid, dim3(NT), stream, a)
@@ -410,6 +364,36 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
             case 4: e = launch_pdl(dispatch_bf16_kernel<4>, grid, dim3(NT), 0, stream, a); break;
             case 8: e = launch_pdl(dispatch_bf16_kernel<8>, grid, dim3(NT), 0, stream, a); break;
             default: e = launch_pdl(dispatch_bf16_kernel<16>, grid, dim3(NT), 0, stream, a); break;
+        }
+    }
+    return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+int launch_shard_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
+                          const float* smooth, const ShardTable& tab, cudaStream_t stream) {
+    if (s.B == 0) return EP_OK;
+    DispatchArgs a = make_dispatch_args(s, p, x, smooth, nullptr, nullptr);
+    a.self_rows = 0;
+    int U = 0, NT = 0;
+    cudaError_t e = cudaSuccess;
+    const dim3 grid(s.B);
+    if (s.quant_mode != 0) {
+        if (pick_units(s.d / 16, 8, &U, &NT) != EP_OK) return EP_ERR_UNSUPPORTED;
+        const bool st = s.quant_mode == 1;
+        switch (U) {
+            case 1: e = launch_pdl(st ? dispatch_int8_shard_kernel<1, true> : dispatch_int8_shard_kernel<1, false>, grid, dim3(NT), 0, stream, a, tab); break;
+            case 2: e = launch_pdl(st ? dispatch_int8_shard_kernel<2, true> : dispatch_int8_shard_kernel<2, false>, grid, dim3(NT), 0, stream, a, tab); break;
+            case 4: e = launch_pdl(st ? dispatch_int8_shard_kernel<4, true> : dispatch_int8_shard_kernel<4, false>, grid, dim3(NT), 0, stream, a, tab); break;
+            default: e = launch_pdl(st ? dispatch_int8_shard_kernel<8, true> : dispatch_int8_shard_kernel<8, false>, grid, dim3(NT), 0, stream, a, tab); break;
+        }
+    } else {
+        if (pick_units(s.d / 8, 16, &U, &NT) != EP_OK) return EP_ERR_UNSUPPORTED;
+        switch (U) {
+            case 1: e = launch_pdl(dispatch_bf16_shard_kernel<1>, grid, dim3(NT), 0, stream, a, tab); break;
+            case 2: e = launch_pdl(dispatch_bf16_shard_kernel<2>, grid, dim3(NT), 0, stream, a, tab); break;
+            case 4: e = launch_pdl(dispatch_bf16_shard_kernel<4>, grid, dim3(NT), 0, stream, a, tab); break;
+            case 8: e = launch_pdl(dispatch_bf16_shard_kernel<8>, grid, dim3(NT), 0, stream, a, tab); break;
+            default: e = launch_pdl(dispatch_bf16_shard_kernel<16>, grid, dim3(NT), 0, stream, a, tab); break;
         }
     }
     return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;

@@ -185,6 +185,152 @@ int ep_buffer_check(ep_buffer* buf, ep_stream_t stream, uint32_t* err_bits) {
     return EP_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Multi-GPU forms (one process per logical rank).
+// ---------------------------------------------------------------------------
+namespace {
+
+// Shard workspace: the layout workspace of this rank's tokens laid out as a one-rank
+// problem (header and, above 256 tokens, the chunk counts), then the layout's
+// expert_count [E_tot] and expert_offset [E_tot + 1] scratch.
+struct ShardWs {
+    size_t layout_bytes, count_off, offset_off, total;
+};
+
+int shard_local(const ep_config* cfg, ep::Shape* ls, ShardWs* ws) {
+    const int st = check_config(cfg);
+    if (st != EP_OK) return st;
+    if (cfg->layout != 0 || cfg->smooth_rows > 1 || cfg->P > EP_SHARD_MAX_RANKS) return EP_ERR_UNSUPPORTED;
+    ep::Shape s = ep::make_shape(*cfg);  // global rows E * P * M
+    s.B = s.T;                           // this rank's tokens
+    s.P = 1;                             // laid out as a one-rank problem (global rows via gstride)
+    *ls = s;
+    ws->layout_bytes = ep::workspace_bytes(s);
+    ws->count_off = ws->layout_bytes;
+    ws->offset_off = ws->count_off + 4 * (size_t)s.E_tot;
+    ws->total = (ws->offset_off + 4 * ((size_t)s.E_tot + 1) + 255) & ~(size_t)255;
+    return EP_OK;
+}
+
+int shard_table(const ep_config* cfg, const ep_shard_table* tab, bool combine, ep::ShardTable* out) {
+    if (!tab || tab->rank < 0 || tab->rank >= cfg->P) return EP_ERR_INVALID_ARG;
+    for (int q = 0; q < cfg->P; ++q) {
+        if (!tab->recv_x[q] || !aligned16(tab->recv_x[q])) return EP_ERR_INVALID_ARG;
+        if (!combine && cfg->quant_mode == 2 && (!tab->recv_scale[q] || !aligned4(tab->recv_scale[q])))
+            return EP_ERR_INVALID_ARG;
+        if (!combine && tab->recv_src[q] && !aligned4(tab->recv_src[q])) return EP_ERR_INVALID_ARG;
+        out->x[q] = tab->recv_x[q];
+        out->scale[q] = combine ? nullptr : tab->recv_scale[q];
+        out->src[q] = combine ? nullptr : tab->recv_src[q];
+    }
+    for (int q = cfg->P; q < EP_SHARD_MAX_RANKS; ++q) {
+        out->x[q] = nullptr;
+        out->scale[q] = nullptr;
+        out->src[q] = nullptr;
+    }
+    out->slab_rows = (long long)(cfg->E / cfg->P) * cfg->P * cfg->M;
+    out->token_base = tab->rank * (cfg->B / cfg->P);
+    return EP_OK;
+}
+
+}  // namespace
+
+int ep_shard_workspace_size(const ep_config* cfg, size_t* bytes) {
+    if (!bytes) return EP_ERR_INVALID_ARG;
+    ep::Shape ls;
+    ShardWs ws;
+    const int st = shard_local(cfg, &ls, &ws);
+    if (st != EP_OK) return st;
+    *bytes = ws.total;
+    return EP_OK;
+}
+
+int ep_shard_layout(const ep_config* cfg, int32_t rank, const int32_t* topk_idx,
+                    const uint8_t* x_active_mask, int32_t* dst_pos, int32_t* send_count,
+                    void* workspace, ep_stream_t stream) {
+    ep::Shape ls;
+    ShardWs ws;
+    const int st = shard_local(cfg, &ls, &ws);
+    if (st != EP_OK) return st;
+    if (rank < 0 || rank >= cfg->P) return EP_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace) || !send_count || !aligned4(send_count)) return EP_ERR_INVALID_ARG;
+    if (ls.B > 0 && (!topk_idx || !aligned4(topk_idx) || !dst_pos || !aligned4(dst_pos)))
+        return EP_ERR_INVALID_ARG;
+    ep_buffer_ptrs p = {};
+    char* w = static_cast<char*>(workspace);
+    p.expert_count = reinterpret_cast<int32_t*>(w + ws.count_off);
+    p.expert_offset = reinterpret_cast<int32_t*>(w + ws.offset_off);
+    p.recv_count = send_count;  // [E][1]: this rank's column
+    p.dst_pos = dst_pos;
+    p.recv_src = nullptr;       // written by the dispatch, into the owners' slabs
+    p.workspace = workspace;
+    return ep::launch_layout(ls, p, topk_idx, x_active_mask, reinterpret_cast<cudaStream_t>(stream),
+                             cfg->P * cfg->M, rank * cfg->M);
+}
+
+int ep_shard_dispatch(const ep_config* cfg, const ep_shard_table* tab, const uint16_t* x,
+                      const float* smooth_scale, const int32_t* dst_pos, float* token_scale,
+                      void* workspace, ep_stream_t stream) {
+    ep::Shape ls;
+    ShardWs ws;
+    int st = shard_local(cfg, &ls, &ws);
+    if (st != EP_OK) return st;
+    ep::ShardTable t;
+    st = shard_table(cfg, tab, false, &t);
+    if (st != EP_OK) return st;
+    if (!workspace || !aligned16(workspace)) return EP_ERR_INVALID_ARG;
+    if (ls.B > 0 && (!x || !aligned16(x) || !dst_pos || !aligned4(dst_pos))) return EP_ERR_INVALID_ARG;
+    if (ls.B > 0 && cfg->quant_mode == 2 && (!token_scale || !aligned4(token_scale))) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && (cfg->smooth_rows == 0 || cfg->quant_mode == 0 || !aligned16(smooth_scale)))
+        return EP_ERR_INVALID_ARG;
+    ep_buffer_ptrs p = {};
+    p.dst_pos = const_cast<int32_t*>(dst_pos);
+    p.token_scale = token_scale;
+    p.workspace = workspace;
+    return ep::launch_shard_dispatch(ls, p, x, smooth_scale, t, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ep_shard_combine(const ep_config* cfg, const ep_shard_table* tab, const int32_t* topk_idx,
+                     const float* topk_weights, const uint8_t* x_active_mask, const int32_t* dst_pos,
+                     const uint16_t* ori_x, const uint16_t* a1, const uint16_t* a2, const uint16_t* v,
+                     uint16_t* y, void* workspace, ep_stream_t stream) {
+    ep::Shape ls;
+    ShardWs ws;
+    int st = shard_local(cfg, &ls, &ws);
+    if (st != EP_OK) return st;
+    ep::ShardTable t;
+    st = shard_table(cfg, tab, true, &t);
+    if (st != EP_OK) return st;
+    if (!workspace || !aligned16(workspace)) return EP_ERR_INVALID_ARG;
+    if (ls.B > 0) {
+        if (!topk_idx || !aligned4(topk_idx) || !topk_weights || !aligned4(topk_weights) || !dst_pos ||
+            !aligned4(dst_pos))
+            return EP_ERR_INVALID_ARG;
+        if (!y || !aligned16(y)) return EP_ERR_INVALID_ARG;
+        if (cfg->n_copy + cfg->n_const > 0 && (!ori_x || !aligned16(ori_x))) return EP_ERR_INVALID_ARG;
+        if (cfg->n_const > 0 && (!a1 || !a2 || !v || !aligned16(a1) || !aligned16(a2) || !aligned16(v)))
+            return EP_ERR_INVALID_ARG;
+        if (y == ori_x) return EP_ERR_INVALID_ARG;
+    }
+    ep_buffer_ptrs p = {};
+    p.dst_pos = const_cast<int32_t*>(dst_pos);
+    p.workspace = workspace;
+    return ep::launch_shard_combine(ls, p, topk_idx, topk_weights, x_active_mask, ori_x, a1, a2, v, y, t,
+                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ep_shard_check(void* workspace, ep_stream_t stream, uint32_t* err_bits) {
+    if (!workspace || !err_bits) return EP_ERR_INVALID_ARG;
+    auto* hdr = reinterpret_cast<ep::WsHeader*>(workspace);
+    unsigned host = 0;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaMemcpy(&host, &hdr->err, sizeof host, cudaMemcpyDeviceToHost) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaMemset(&hdr->err, 0, sizeof host) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return EP_ERR_CUDA;
+    *err_bits = host;
+    return EP_OK;
+}
+
 const char* ep_status_str(int status) {
     switch (status) {
         case EP_OK: return "ok";

@@ -25,6 +25,16 @@ constexpr int kMaxD = 32768;     // 256 threads x 8 units of 16 elements
 
 constexpr int kMaxPackedEP = 24576;  // E * P of the packed layout (the pack kernel's shared table)
 
+// Receive slabs of the ranks of a multi-GPU run (a kernel parameter): slab q holds
+// the slab_rows = L * P * M low-latency rows of experts q*L .. q*L+L-1.
+struct ShardTable {
+    void* x[EP_SHARD_MAX_RANKS];        // recv_x slabs (dispatch) or expert-output slabs (combine)
+    float* scale[EP_SHARD_MAX_RANKS];   // recv_scale slabs (dispatch, quant_mode 2)
+    int32_t* src[EP_SHARD_MAX_RANKS];   // recv_src slabs (dispatch; may be null)
+    long long slab_rows;
+    int token_base;                     // global index of this rank's first token
+};
+
 struct Shape {
     int B, d, k, P, M, E, Z, C, K, T, L, E_tot, n_special;
     int quant_mode;     // 0 bf16, 1 static int8, 2 dynamic int8
@@ -62,8 +72,9 @@ inline size_t workspace_bytes(const Shape& s) {
 // Host launchers (one per kernel family); each returns an EP_* status.
 // active: x_active_mask [B] (nonzero = active) or null; an inactive token takes no
 // part (as if every pick were -1).
+// gstride / rbase: see LayoutArgs (default: gstride = P * M, rbase = 0).
 int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
-                  const uint8_t* active, cudaStream_t stream);
+                  const uint8_t* active, cudaStream_t stream, int gstride = -1, int rbase = 0);
 // topk_idx: the routing of the latest layout on this buffer (lets dispatch derive
 // its receive rows itself for small per-rank batches); may be null, except with a
 // per-expert smooth scale, where it names each copy's expert.
@@ -80,6 +91,15 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
                    const uint16_t* ori_x,
                    const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
                    cudaStream_t stream);
+
+// Multi-GPU forms (one process per logical rank; see ShardTable).  s is the local
+// view: B = T tokens of this rank, rows = the global E * P * M.
+int launch_shard_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
+                          const float* smooth, const ShardTable& tab, cudaStream_t stream);
+int launch_shard_combine(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
+                         const float* topk_weights, const uint8_t* active, const uint16_t* ori_x,
+                         const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
+                         const ShardTable& tab, cudaStream_t stream);
 
 // Streaming multiprocessors of the current device (queried once per device).
 inline int num_sms() {
@@ -150,52 +170,18 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return r;
 }
 
+// 16-byte store.  No "memory" clobber: nothing in the library reads back, within
+// the same kernel, what these stores write, so the compiler may keep shared-memory
+// values (row pointers, weights) in registers across the stores.
 __device__ __forceinline__ void st_v4(void* p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y),
-                 "r"(v.z), "r"(v.w)
-                 : "memory");
+                 "r"(v.z), "r"(v.w));
 }
 
-// 32 bytes per thread (sm_100 256-bit global accesses): one load or store moves 16
-// bf16 values, the source of one 16-byte int8 vector.
-struct V8 {
-    uint32_t w[8];
-};
-__device__ __forceinline__ V8 ld_stream_v8(const void* p) {
-    V8 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]),
-                   "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7])
-                 : "l"(p));
-    return r;
-}
-__device__ __forceinline__ void st_v8(void* p, const V8& v) {
-    asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
-                 "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
-                 "r"(v.w[7])
-                 : "memory");
-}
-
-// 32 bytes at p: one 256-bit access when `wide` (the host has checked that every
-// such address is 32-byte aligned), else two 16-byte accesses (the ABI promises
-// only 16-byte alignment, and an int8 row of d % 32 == 16 bytes leaves every
-// other row on a 16-byte boundary).
-__device__ __forceinline__ V8 ld32(const void* p, bool wide) {
-    if (wide) return ld_stream_v8(p);
-    const uint4 a = ld_stream_v4(p);
-    const uint4 b = ld_stream_v4(reinterpret_cast<const char*>(p) + 16);
-    V8 r;
-    r.w[0] = a.x; r.w[1] = a.y; r.w[2] = a.z; r.w[3] = a.w;
-    r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
-    return r;
-}
-__device__ __forceinline__ void st32(void* p, const V8& v, bool wide) {
-    if (wide) {
-        st_v8(p, v);
-    } else {
-        st_v4(p, make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
-        st_v4(reinterpret_cast<char*>(p) + 16, make_uint4(v.w[4], v.w[5], v.w[6], v.w[7]));
-    }
+// Ask the copy engine to bring [p, p + bytes) into L2 (no data returned to the SM;
+// p and bytes 16-byte aligned).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes));
 }
 
 // bf16 bits <-> fp32: a bf16 is the high half of a binary32.
@@ -236,34 +222,27 @@ __device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
     if (all && (int)(threadIdx.x & 31) == __ffs(active) - 1) atomicOr(err_word, all);
 }
 
-// Shared memory of one warp of the warp-per-token kernels: the routing table
-// (E uint16, 16-byte padded); the dispatch kernels may add a staging row after it.
-__host__ __device__ __forceinline__ int warp_tab_bytes(int E) { return ((2 * E + 15) / 16) * 16; }
-
-// Zero this warp's routing table (E uint16) before its first use.
-__device__ __forceinline__ void zero_warp_tab(uint16_t* tab, int E) {
-    uint32_t* w = reinterpret_cast<uint32_t*>(tab);
-    const int n = warp_tab_bytes(E) / 4;
-    for (int i = threadIdx.x & 31; i < n; i += 32) w[i] = 0u;
-    __syncwarp();
-}
-
 // Receive rows of token t derived from the routing alone, for small per-rank
 // batches: the slot of a routed id g is the number of earlier tokens of the same
 // rank that picked g (a token counts once), which is exactly the slot the layout
 // kernels assign; a routed id repeated inside the token gets row -1 after its
 // first occurrence.  Inactive tokens (active[t] == 0, when a mask is given) route
-// nothing and are not counted.  The earlier tokens' ids come from L2.  s_rows,
-// s_g, s_cnt: k-entry shared arrays.  All threads of the CTA call it; on return
-// s_rows[j] is written by thread j (j < k) and not yet published to the other threads.
+// nothing and are not counted.  The earlier tokens' ids come from L2.
+// s_rows, s_g, s_cnt: k-entry shared arrays; tab: E uint16 of shared memory, set
+// here to one bit per routed pick of this token at the pick's expert, so that an
+// earlier token costs k table lookups rather than k * k compares.  All threads of
+// the CTA call it; on return s_rows[j] is written by thread j (j < k) and not yet
+// published to the other threads.
 // Packed rows (expert_offset and recv_count given): the row is expert_offset[g] +
 // sum_{r' < r} recv_count[g][r'] + slot.  Those counts come from the layout kernel,
 // which the caller guarantees complete; they are read through L2 (another grid
 // wrote them).
 __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* active, int t, int k,
                                     int E, int T, int P, int M, int* s_rows, int* s_g, int* s_cnt,
-                                    const int32_t* expert_offset = nullptr,
+                                    uint16_t* tab, const int32_t* expert_offset = nullptr,
                                     const int32_t* recv_count = nullptr) {
+    uint32_t* tw = reinterpret_cast<uint32_t*>(tab);
+    for (int i = threadIdx.x; i < (E + 1) / 2; i += blockDim.x) tw[i] = 0u;
     if (threadIdx.x < k) {
         const int j = threadIdx.x;
         const int g = topk_idx[(size_t)t * k + j];
@@ -274,16 +253,26 @@ __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* acti
         s_cnt[j] = 0;
     }
     __syncthreads();
+    if (threadIdx.x < k && s_g[threadIdx.x] >= 0) tab[s_g[threadIdx.x]] = (uint16_t)(1u << threadIdx.x);
+    __syncthreads();
     const int r = t / T;
+    const bool vec4 = (k % 4 == 0) && ((reinterpret_cast<uintptr_t>(topk_idx) & 15) == 0);
     for (int tt = r * T + (int)threadIdx.x; tt < t; tt += blockDim.x) {
         if (active && !active[tt]) continue;
         const int32_t* ids = topk_idx + (size_t)tt * k;
         unsigned hit = 0;
-        for (int jj = 0; jj < k; ++jj) {
-            const int v = __ldg(ids + jj);
-            for (int j = 0; j < k; ++j) {
-                const int g = s_g[j];
-                if (g >= 0 && v == g) hit |= 1u << j;
+        if (vec4) {
+            for (int j4 = 0; 4 * j4 < k; ++j4) {
+                const int4 v = __ldg(reinterpret_cast<const int4*>(ids) + j4);
+                hit |= (unsigned)v.x < (unsigned)E ? tab[v.x] : 0u;
+                hit |= (unsigned)v.y < (unsigned)E ? tab[v.y] : 0u;
+                hit |= (unsigned)v.z < (unsigned)E ? tab[v.z] : 0u;
+                hit |= (unsigned)v.w < (unsigned)E ? tab[v.w] : 0u;
+            }
+        } else {
+            for (int jj = 0; jj < k; ++jj) {
+                const int v = __ldg(ids + jj);
+                hit |= (unsigned)v < (unsigned)E ? tab[v] : 0u;
             }
         }
         while (hit) {
@@ -310,99 +299,6 @@ __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* acti
         if (g >= 0) row = expert_offset ? s_cnt[threadIdx.x] : g * P * M + r * M + s_cnt[threadIdx.x];
         s_rows[threadIdx.x] = row;
     }
-}
-
-// The same receive rows computed by one warp on its own, for kernels whose warps
-// each own a token (no CTA barrier).  tab: this warp's shared table of E uint16
-// entries, all zero on entry and zero again on return; entry g holds the bit of
-// the pick of this token that routes to g.  An earlier token of the rank looks
-// each of its ids up in the table, so it costs k shared loads instead of k * k
-// compares, and a token counts once per expert however often it repeats an id.
-// On return row[j] is the receive row of pick j (-1: not routed) in every lane.
-template <int KM>
-__device__ __forceinline__ void routing_rows_warp(const int32_t* __restrict__ topk_idx,
-                                                  const uint8_t* active, int t, int k, int E,
-                                                  int T, int P, int M, uint16_t* tab,
-                                                  int (&row)[KM],
-                                                  const int32_t* expert_offset = nullptr,
-                                                  const int32_t* recv_count = nullptr) {
-    static_assert(KM <= 16, "pick bits are kept in 16-bit table entries");
-    const unsigned FULL = 0xffffffffu;
-    const int lane = threadIdx.x & 31;
-    const bool on = !(active && !active[t]);
-    const int mine = lane < k ? __ldg(topk_idx + (size_t)t * k + lane) : -1;
-    int g[KM];
-    unsigned rb = 0;  // routed picks: an id in [0, E), its first occurrence, token active
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        g[j] = __shfl_sync(FULL, mine, j);
-        bool routed = on && j < k && g[j] >= 0 && g[j] < E;
-#pragma unroll
-        for (int jj = 0; jj < j; ++jj)
-            if (g[jj] == g[j]) routed = false;
-        if (routed) rb |= 1u << j;
-    }
-    if ((rb >> lane) & 1u) tab[mine] = (uint16_t)(1u << lane);
-    __syncwarp();
-    const int r = t / T;
-    int cnt[KM];
-#pragma unroll
-    for (int j = 0; j < KM; ++j) cnt[j] = 0;
-    const bool vec4 = (k % 4 == 0) && ((reinterpret_cast<uintptr_t>(topk_idx) & 15) == 0);
-    for (int tt = r * T + lane; tt < t; tt += 32) {
-        if (active && !active[tt]) continue;
-        const int32_t* ids = topk_idx + (size_t)tt * k;
-        unsigned hit = 0;
-        if (vec4) {
-#pragma unroll
-            for (int j4 = 0; j4 < KM / 4; ++j4) {
-                if (4 * j4 >= k) continue;
-                const int4 v = __ldg(reinterpret_cast<const int4*>(ids) + j4);
-                hit |= (unsigned)v.x < (unsigned)E ? tab[v.x] : 0u;
-                hit |= (unsigned)v.y < (unsigned)E ? tab[v.y] : 0u;
-                hit |= (unsigned)v.z < (unsigned)E ? tab[v.z] : 0u;
-                hit |= (unsigned)v.w < (unsigned)E ? tab[v.w] : 0u;
-            }
-        } else {
-#pragma unroll
-            for (int jj = 0; jj < KM; ++jj) {
-                if (jj >= k) continue;
-                const int v = __ldg(ids + jj);
-                hit |= (unsigned)v < (unsigned)E ? tab[v] : 0u;
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < KM; ++j) cnt[j] += (hit >> j) & 1u;
-    }
-#pragma unroll
-    for (int j = 0; j < KM; ++j) cnt[j] = (int)__reduce_add_sync(FULL, (unsigned)cnt[j]);
-    if (expert_offset) {
-        // packed: add expert_offset[g] and the r lower ranks' counts of g
-        const int per = r + 1;
-        int part[KM];
-#pragma unroll
-        for (int j = 0; j < KM; ++j) part[j] = 0;
-        for (int i = lane; i < k * per; i += 32) {
-            const int jsel = i / per, rr = i - jsel * per;
-            int gsel = -1;
-#pragma unroll
-            for (int j = 0; j < KM; ++j)
-                if (j == jsel && ((rb >> j) & 1u)) gsel = g[j];
-            if (gsel < 0) continue;
-            const int val = rr < r ? __ldcg(recv_count + (size_t)gsel * P + rr) : __ldcg(expert_offset + gsel);
-#pragma unroll
-            for (int j = 0; j < KM; ++j)
-                if (j == jsel) part[j] += val;
-        }
-#pragma unroll
-        for (int j = 0; j < KM; ++j) cnt[j] += (int)__reduce_add_sync(FULL, (unsigned)part[j]);
-    }
-    __syncwarp();
-    if ((rb >> lane) & 1u) tab[mine] = 0;
-    __syncwarp();
-#pragma unroll
-    for (int j = 0; j < KM; ++j)
-        row[j] = ((rb >> j) & 1u) ? (expert_offset ? cnt[j] : g[j] * P * M + r * M + cnt[j]) : -1;
 }
 
 }  // namespace ep

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kChunkTokens) layout_chunk_rows_kernel(LayoutA
             const int g = ids[j];
             int row = -1;
             if (ep_in_range(g, E, &a.ws->err)) {
-                row = g * a.P * a.M + r * a.M + pre[g] + slot;
+                row = g * a.gstride + r * a.M + a.rbase + pre[g] + slot;
                 if (!ep_in_range(row, a.rows, &a.ws->err)) row = -1;
                 else if (a.recv_src) a.recv_src[row] = t;
             }
@@ -220,7 +220,8 @@ __global__ void __launch_bounds__(256) layout_pack_kernel(const int32_t* expert_
 }  // namespace
 
 int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
-                  const uint8_t* active, cudaStream_t stream) {
+                  const uint8_t* active, cudaStream_t stream, int gstride, int rbase) {
+    if (gstride < 0) gstride = s.P * s.M;
     if (s.layout == 1 && s.B > 0) {
         // counts and low-latency-form rows (stride T, no recv_src), then pack
         Shape ll = s;
@@ -290,6 +291,8 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
         a1.n_special = s.n_special; a1.E_tot = s.E_tot;
         a1.rows = s.rows;
         a1.warps = 8;
+        a1.gstride = gstride;
+        a1.rbase = rbase;
         const int ranks_per_cta = 8 / cpr;
         const int grid = 1 + (s.P + ranks_per_cta - 1) / ranks_per_cta;
         cudaError_t e;
@@ -334,6 +337,8 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
     a.n_special = s.n_special; a.E_tot = s.E_tot;
     a.rows = s.rows;
     a.warps = kChunkTokens / 32;
+    a.gstride = gstride;
+    a.rbase = rbase;
     const dim3 grid((unsigned)n_chunks, (unsigned)s.P), block(kChunkTokens);
     cudaError_t e;
     if (s.k <= 2)
@@ -369,7 +374,7 @@ int launch_layout(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_i
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr size_t kStaticScratchBytes = 64 * 1024;  // 256-byte header + P*(Z+C+K) int32 counts
+constexpr size_t kStaticScratchBytes = 64 * 1024;  // 256-byte header + P*ceil(T/256)*(E+Z+C+K) int32 chunk counts when T > 256
 
 // Lives on every GPU that loads this library, until the process exits.
 static __device__ __align__(256) unsigned char g_layout_scratch[kStaticScratchBytes];

@@ -21,6 +21,10 @@ struct LayoutArgs {
     int B, k, P, M, E, T, n_special, E_tot;
     long long rows;       // receive rows the computed row ids index (E * P * M)
     int warps;            // warps per CTA
+    // row of (expert g, rank r, slot) = g * gstride + r * M + rbase + slot: P * M and 0
+    // on one GPU; a process that lays out only its own rank's tokens (P = 1 here)
+    // uses the global stride and its rank's offset
+    int gstride, rbase;
 };
 
 // Exclusive prefix of cnt[0..n) into out[0..n], out[n] = total; all threads of the
@@ -214,7 +218,7 @@ __device__ __forceinline__ void layout_small_body(const LayoutArgs& a, int cpr, 
                 const int g = ids[j];
                 int before = 0;  // the rank's tokens in its earlier chunks that routed to g
                 for (int cc = 0; cc < c; ++cc) before += __popc(rank_masks[(size_t)cc * E + g]);
-                row = g * P * a.M + r * a.M + before + __popc(my_mask[g] & lt);
+                row = g * a.gstride + r * a.M + a.rbase + before + __popc(my_mask[g] & lt);
                 if (!ep_in_range(row, a.rows, &a.ws->err)) row = -1;
                 else if (a.recv_src) a.recv_src[row] = t;
             }

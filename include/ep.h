@@ -212,7 +212,13 @@ EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, const uint8_t* x_a
  * passed to that ep_layout (which must still hold the same values) instead of reading dst_pos,
  * so it can run alongside the layout kernel (for the packed layout, alongside its
  * second kernel, reading the per-expert counts the first one wrote); it finishes
- * only after the layout kernels have.  Call it on the stream of that ep_layout, after it. */
+ * only after the layout kernels have.  Call it on the stream of that ep_layout, after it.
+ * Ordering: in that small-batch form the kernel reads x and the routing and writes
+ * recv_x, recv_scale and token_scale before it waits for the kernel ahead of it on
+ * the stream.  That is safe because ep_layout's kernel waits for everything before
+ * it first.  So no kernel that is launched with programmatic dependent launch and
+ * triggers its dependents early may sit between ep_layout and ep_dispatch on the
+ * stream (ordinary launches, copies and event waits may). */
 EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale,
                 ep_stream_t stream);
 
@@ -235,7 +241,14 @@ EP_API int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx,
  * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos,
  * or for T = B/P <= 128 derives the same rows from topk_idx (which must hold the
  * ids given to that layout) and the layout's counts.
- * y must not overlap any input. */
+ * y must not overlap any input.
+ * Ordering: in that small-batch form the kernel reads topk_idx, x_active_mask and
+ * (packed layout) expert_offset and recv_count before it waits for the kernel
+ * ahead of it on the stream, and reads expert outputs and writes y only after.
+ * The library's own kernels before it (ep_layout, ep_dispatch) let it start only
+ * once those counts are final.  A kernel launched with programmatic dependent
+ * launch that triggers its dependents early and writes topk_idx, the mask or
+ * those counts must not be the one right before ep_combine on the stream. */
 EP_API int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,
                const float* topk_weights, const uint8_t* x_active_mask, const uint16_t* ori_x,
                const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
@@ -276,6 +289,77 @@ EP_API int ep_layout_static_scratch(const ep_config* cfg, const int32_t* topk_id
 
 /* Synchronize `stream`, read the device error word into *err_bits and clear it. */
 EP_API int ep_buffer_check(ep_buffer* buf, ep_stream_t stream, uint32_t* err_bits);
+
+/*
+ * ---------------------------------------------------------------------------
+ * Expert parallelism across GPUs: one process per GPU (the wide expert
+ * parallelism of the Wide-EP blog (getimpala.ai), sections on wide EP and DBO; the
+ * low-latency layout of DeepEP issue #84, where each rank's receive buffer holds
+ * [local_experts][ranks * max_tokens][hidden]).
+ *
+ * Logical rank r is one process.  It holds its own T = B / P tokens (x, topk_idx,
+ * topk_weights and x_active_mask of global tokens r*T .. r*T+T-1, indexed locally
+ * 0 .. T-1) and receive slab r: the low-latency rows of its experts r*L .. r*L+L-1,
+ * [L][P*M][d], slab row = global row - r*L*P*M, where the global row of (expert g,
+ * source rank r, slot) is g*P*M + r*M + slot exactly as on one GPU.  A sender
+ * therefore places its tokens with no information from other ranks:
+ *   ep_shard_layout    its picks' global rows (dst_pos [T][k]) and send_count [E],
+ *                      its routed picks per expert: entries q*L .. q*L+L-1 are
+ *                      column r of rank q's recv_count [L][P];
+ *   (count exchange)   done by the caller, e.g. one all-to-all of send_count;
+ *   ep_shard_dispatch  quantizes its tokens (as ep_dispatch) and stores every routed
+ *                      copy straight into the owning rank's slab, with the row's
+ *                      recv_scale and recv_src (global token index);
+ *   ep_shard_combine   reads each routed pick's expert output from the owning
+ *                      rank's slab and reduces as ep_combine into y [T][d].
+ * The slabs are reached through an ep_shard_table of device addresses: this
+ * process's own slab and the peers' slabs mapped into it (CUDA IPC; every access is
+ * a plain load or store over NVLink, no bulk or multicast copy), or, on one GPU,
+ * P separate allocations.  Between a rank's dispatch and another rank's reads of
+ * its slab the caller orders the GPUs (e.g. a collective or a barrier on the
+ * stream); the library itself never waits on another rank.
+ * Low-latency layout (layout 0) only; smooth_rows 0 or 1; P <= EP_SHARD_MAX_RANKS.
+ */
+#define EP_SHARD_MAX_RANKS 64
+
+typedef struct {
+    int32_t rank;                           /* this process's logical rank, 0 <= rank < P */
+    void* recv_x[EP_SHARD_MAX_RANKS];       /* [P] device address of rank q's slab: recv_x rows
+                                               [L*P*M][d] (int8, or bf16 in quant_mode 0) for
+                                               ep_shard_dispatch; bf16 expert outputs of the same
+                                               rows for ep_shard_combine */
+    float* recv_scale[EP_SHARD_MAX_RANKS];  /* [P] recv_scale slabs [L*P*M] (quant_mode 2, dispatch) */
+    int32_t* recv_src[EP_SHARD_MAX_RANKS];  /* [P] recv_src slabs [L*P*M] (dispatch); NULL = not written */
+} ep_shard_table;
+
+/* Bytes of the device workspace of the ep_shard_* calls (one per process; the caller
+ * allocates it and zero-fills it once before the first call). */
+EP_API int ep_shard_workspace_size(const ep_config* cfg, size_t* bytes);
+
+/* Layout of rank `rank`'s T tokens (topk_idx int32 [T][k], x_active_mask uint8 [T] or
+ * NULL): dst_pos int32 [T][k] (global low-latency rows, -1 if not routed) and
+ * send_count int32 [E].  Error bits go to the workspace (ep_shard_check). */
+EP_API int ep_shard_layout(const ep_config* cfg, int32_t rank, const int32_t* topk_idx,
+                           const uint8_t* x_active_mask, int32_t* dst_pos, int32_t* send_count,
+                           void* workspace, ep_stream_t stream);
+
+/* Dispatch of rank tab->rank's tokens x (bf16 [T][d]) to the rows dst_pos of its
+ * ep_shard_layout, into the slabs of `tab` (recv_x, recv_scale in quant_mode 2, recv_src
+ * = rank*T + local token).  token_scale: fp32 [T] (quant_mode 2), else NULL. */
+EP_API int ep_shard_dispatch(const ep_config* cfg, const ep_shard_table* tab, const uint16_t* x,
+                             const float* smooth_scale, const int32_t* dst_pos, float* token_scale,
+                             void* workspace, ep_stream_t stream);
+
+/* Combine of rank tab->rank's tokens into y (bf16 [T][d]); tab->recv_x[q] are the bf16
+ * expert-output slabs; other arguments as ep_combine, local to this rank. */
+EP_API int ep_shard_combine(const ep_config* cfg, const ep_shard_table* tab,
+                            const int32_t* topk_idx, const float* topk_weights,
+                            const uint8_t* x_active_mask, const int32_t* dst_pos,
+                            const uint16_t* ori_x, const uint16_t* a1, const uint16_t* a2,
+                            const uint16_t* v, uint16_t* y, void* workspace, ep_stream_t stream);
+
+/* Synchronize `stream`, read the shard workspace's error word into *err_bits, clear it. */
+EP_API int ep_shard_check(void* workspace, ep_stream_t stream, uint32_t* err_bits);
 
 /* Static text for a status code. */
 EP_API const char* ep_status_str(int status);
