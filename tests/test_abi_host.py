@@ -167,3 +167,58 @@ def test_product_path_has_no_oracle_import():
                 bad = re.search(r"^\s*(import oracle|from oracle)|libep_oracle|orc_[a-z]+\(", text,
                                 flags=re.M)
                 assert not bad, os.path.join(dirpath, f)
+
+
+def test_shard_workspace_size_and_unsupported_forms():
+    # one rank's layout workspace (header + counts scratch), 256-byte granular
+    n = abi.ep_shard_workspace_size(cfg())
+    assert n % 256 == 0 and n >= 256 + 4 * (2 * 256 + 1)
+    # above 256 tokens per rank the chunk counts of the rank's own tokens are added
+    big = abi.ep_shard_workspace_size(cfg(B=8 * 1024, M=1024))
+    assert big >= n + 4 * 4 * 256
+    for kw, status in ((dict(layout=1), abi.EP_ERR_UNSUPPORTED),
+                       (dict(smooth_rows=256), abi.EP_ERR_UNSUPPORTED),
+                       (dict(P=128, E=256, B=128, M=1), abi.EP_ERR_UNSUPPORTED),
+                       (dict(B=7), abi.EP_ERR_INVALID_ARG)):
+        with pytest.raises(abi.EPError) as ei:
+            abi.ep_shard_workspace_size(cfg(**kw))
+        assert ei.value.status == status, kw
+
+
+def test_shard_calls_reject_bad_arguments_before_cuda():
+    c = cfg()
+    fake = 1 << 40  # 16-byte aligned, never dereferenced: validation fails first
+    good = abi.make_shard_table(0, [fake] * 8, [fake] * 8, [fake] * 8)
+    # rank out of range
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_layout(c, 8, fake, None, fake, fake, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    # a missing slab in the table
+    holes = abi.make_shard_table(0, [fake] * 7 + [None], [fake] * 8, [fake] * 8)
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_dispatch(c, holes, fake, None, fake, fake, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    # a misaligned slab
+    odd = abi.make_shard_table(0, [fake + 8] + [fake] * 7, [fake] * 8, [fake] * 8)
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_dispatch(c, odd, fake, None, fake, fake, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    # quant_mode 2 needs the scale slabs and token_scale
+    no_scale = abi.make_shard_table(0, [fake] * 8, None, [fake] * 8)
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_dispatch(c, no_scale, fake, None, fake, fake, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_dispatch(c, good, fake, None, fake, None, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    # combine: y must be given and must not be ori_x
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_combine(c, good, fake, fake, None, fake, None, None, None, None, None, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    # no workspace
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_layout(c, 0, fake, None, fake, fake, None)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_check(None)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
