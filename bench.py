@@ -13,7 +13,8 @@ dequantized receive rows), since the expert computation is not part of
 dispatch/combine.  Up to three buffer sets are used in rotation, so consecutive
 steps touch disjoint memory (more than the 126 MB L2 per step); when only one
 set fits, L2 is flushed (a 512 MB memset) between steps, outside the events.
-Per-kernel durations come from graphs of back-to-back launches of each kernel.
+Per-kernel durations: isolated (one launch after an L2 read-flush, CUDA events
+around it; the roofline figure) and overlapped (graphs of back-to-back launches).
 
 Prints one JSON line (rank 0).  value = algorithmic HBM bytes of the three
 kernels / step time, whole job (all ranks), in GB/s.
@@ -195,6 +196,14 @@ def measured_peak():
         return float(j["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def trimmed_mean(xs, trim=0.1):
+    """Mean of xs without the lowest and highest `trim` fraction."""
+    xs = sorted(xs)
+    n = int(len(xs) * trim)
+    xs = xs[n:len(xs) - n] if len(xs) > 2 * n else xs
+    return sum(xs) / len(xs)
 
 
 def source_hash(name):
@@ -529,32 +538,39 @@ class Workbench:
     _rf_out = None
 
     def isolated_times(self, reps, keys=("layout", "dispatch", "combine", "layout_dispatch")):
-        """Per-launch milliseconds of each kernel run in isolation: every launch is
-        preceded by read_flush(), so it starts on a clean L2 with its inputs in DRAM
-        and overlaps no other launch of the library; graphs of S such pairs are
-        replayed, and the same graph with the reads alone is timed and subtracted."""
-        def graph(names):
-            def body():
-                for i in range(self.S):
+        """Per-launch milliseconds of each library call run alone: read_flush() (L2
+        holds only clean lines of another buffer, the inputs are in DRAM), a CUDA
+        event, the one call, a CUDA event; eager launches, so the call neither
+        overlaps nor follows another launch of the library.  The median over `reps`
+        such launches per call (buffer sets in rotation), as a trimmed mean: event
+        times come in steps of about 1 us on this GPU, and the mean of many jittered
+        samples resolves below the step where a median would sit on it.  The span
+        between the events also holds the processing of the two event records:
+        event_pair is the same measurement with nothing between the events, and it
+        is subtracted (the difference follows ncu's gpu__time_duration of the same
+        launches to within about 0.5 us); raw keeps the spans as measured."""
+        import torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+
+        def timed(name):
+            with torch.cuda.stream(self.stream):
+                for i in range(reps):
                     p, d = self.sets[i % self.R]
                     self.read_flush()
-                    for name in names:
+                    ev[i][0].record(self.stream)
+                    if name:
                         getattr(p, name)(d, self.stream)
-            return self.capture(body)
-        n = max(1, reps // self.S)
-        fg = graph(())
-        self.replay(fg, 1)
-        out = {}
-        for key in keys:
-            g = graph([key])
-            self.replay(g, 1)
-            # alternate kernel and flush-only replays so clock drift hits both alike
-            tk, tf = [], []
-            for _ in range(3):
-                tk.append(self.replay(g, n) / (n * self.S))
-                tf.append(self.replay(fg, n) / (n * self.S))
-            out[key] = statistics.median(tk) - statistics.median(tf)
-        return out, n
+                    ev[i][1].record(self.stream)
+            self.stream.synchronize()
+            return trimmed_mean([a.elapsed_time(b) for a, b in ev])
+
+        timed("layout")  # warm-up
+        raw = {key: timed(key) for key in keys}
+        pair = timed(None)
+        out = {key: max(v - pair, 0.0) for key, v in raw.items()}
+        out["event_pair"] = pair
+        out["raw"] = raw
+        return out
 
     def kernel_times(self, launches):
         """Per-launch milliseconds of each kernel and of the one-call layout+dispatch,
@@ -657,6 +673,7 @@ def run_ours(args):
     step_ms = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(n_lat)]
 
     kern_ms, n_rep = wb.kernel_times(K)
+    iso_ms = wb.isolated_times(min(max(K, 30), 200))
     t_wall2 = time.perf_counter()
     clocks.mark(t_wall0, t_wall2)
     time.sleep(0.03)
@@ -669,14 +686,18 @@ def run_ours(args):
     value = job_bytes / job_s / 1e9
 
     peak, peak_kind = measured_peak()
+    # per kernel: isolated (one launch alone after an L2 read-flush, events around it;
+    # the figure the roofline uses) and overlapped (graphs of back-to-back launches,
+    # where a launch may start while the previous one drains: throughput, not latency)
     kernels = {}
-    tot = sum(kern_ms[n] for n in ("layout", "dispatch", "combine"))
+    tot = sum(iso_ms[n] for n in ("layout", "dispatch", "combine"))
     for name in ("layout", "dispatch", "combine"):
-        ms = kern_ms[name]
+        ms = iso_ms[name]
         ach = wb.kbytes[name] / (ms * 1e-3) / 1e9
         kernels[name] = {"us": 1e3 * ms, "bytes": wb.kbytes[name], "achieved_gbs": ach,
                          "frac_of_measured": ach / peak, "frac_of_8tbs": ach / SPEC_HBM_GBS,
-                         "share": ms / tot}
+                         "share": ms / tot, "us_overlapped": 1e3 * kern_ms[name],
+                         "achieved_gbs_overlapped": wb.kbytes[name] / (kern_ms[name] * 1e-3) / 1e9}
     dom = max(("dispatch", "combine", "layout"), key=lambda n: kernels[n]["share"])
     traffic = recorded_traffic(w.name, dom)
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["achieved_gbs"], "peak": peak,
@@ -685,7 +706,13 @@ def run_ours(args):
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "frac_of_8tbs_spec": kernels[dom]["achieved_gbs"] / SPEC_HBM_GBS,
                 "algorithmic_bytes": wb.kbytes[dom],
-                "duration": "CUDA events around graphs of %d back-to-back launches, %d replays" % (S, n_rep)}
+                "duration": "isolated: trimmed mean over single eager launches, each after a read of a buffer "
+                            "three times the L2 size, of the span between CUDA events around the launch, "
+                            "minus the span of an empty event pair (%.2f us); raw span %.2f us"
+                            % (1e3 * iso_ms["event_pair"], 1e3 * iso_ms["raw"][dom]),
+                "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of this "
+                                "kernel (per launch), recorded in profiles/traffic.json; null once the "
+                                "kernel source has changed since"}
 
     # end to end through the public API with host buffers (eager calls, no graph).
     # Every step uploads its inputs from pinned host memory and reads its y back.
@@ -796,6 +823,7 @@ def run_ours(args):
         "kernels": kernels,
         "layout_then_dispatch_us": 1e3 * kern_ms["layout+dispatch"],
         "layout_dispatch_one_call_us": 1e3 * kern_ms["layout_dispatch"],
+        "layout_dispatch_one_call_us_isolated": 1e3 * iso_ms["layout_dispatch"],
         "comm_gbs_dispatch": wb.n_routed * w.d * (1 if w.quant_mode != 0 else 2)
         / (kern_ms["dispatch"] * 1e-3) / 1e9,
         "roofline": roofline,
@@ -806,6 +834,7 @@ def run_ours(args):
         "gpu_launches": lps * K,
         "gpu_launches_latency_loop": lps * n_lat,
         "gpu_launches_kernel_loops": (5 + lps) * n_rep * S,
+        "gpu_launches_isolated": 5 * min(max(K, 30), 200),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -851,6 +880,7 @@ def run_sweep(args, device):
             wb.replay(fg, 1)
             step_ms -= wb.replay(fg, n) / (n * wb.S)
         kern_ms, _ = wb.kernel_times(steps)
+        iso_ms = wb.isolated_times(min(steps, 100))
         for p, _ in wb.sets:
             assert p.buf.check(stream) == 0
         rec = {"workload": name, "B": w.B, "T": w.T, "P": w.P, "d": w.d, "E": w.E, "k": w.k,
@@ -859,9 +889,13 @@ def run_sweep(args, device):
                "tokens_per_s": w.B / (step_ms * 1e-3), "bytes": wb.kbytes,
                "layout_dispatch_one_call_us": 1e3 * kern_ms["layout_dispatch"]}
         for k in ("layout", "dispatch", "combine"):
-            rec[k + "_us"] = 1e3 * kern_ms[k]
-            rec[k + "_gbs"] = wb.kbytes[k] / (kern_ms[k] * 1e-3) / 1e9
+            rec[k + "_us"] = 1e3 * iso_ms[k]
+            rec[k + "_gbs"] = wb.kbytes[k] / (iso_ms[k] * 1e-3) / 1e9
             rec[k + "_frac_of_measured"] = rec[k + "_gbs"] / peak
+            rec[k + "_us_overlapped"] = 1e3 * kern_ms[k]
+        rec["event_pair_us"] = 1e3 * iso_ms["event_pair"]
+        rec["raw_span_us"] = {k: 1e3 * v for k, v in iso_ms["raw"].items()}
+        rec["layout_dispatch_one_call_us_isolated"] = 1e3 * iso_ms["layout_dispatch"]
         results.append(rec)
         print("%-18s T=%-5d step %8.1f us %7.0f GB/s | layout %7.1f us | dispatch %8.1f us %6.0f GB/s | "
               "combine %8.1f us %6.0f GB/s" % (name, w.T, rec["step_us"], rec["step_gbs"], rec["layout_us"],
