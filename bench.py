@@ -66,6 +66,10 @@ def parse_args(argv=None):
     p.add_argument("--sweep", default=None,
                    help="comma-separated workloads or 'all': per-workload table instead of the JSON line")
     p.add_argument("--sweep-out", default=None, help="where --sweep writes its JSON document")
+    p.add_argument("--profile-launches", type=int, default=0, metavar="N",
+                   help="for profiler captures: build --workload with one buffer set and run N times each "
+                        "of ep_layout, ep_dispatch, ep_layout_dispatch and ep_combine, each after an L2 "
+                        "read-flush; prints no JSON line")
     return p.parse_args(argv)
 
 
@@ -611,6 +615,8 @@ def run_ours(args):
     ep_build.build()
     if args.sweep:
         return run_sweep(args, device)
+    if args.profile_launches:
+        return run_profile_launches(args, device)
 
     w = wl.get(args.workload)
     inp = wl.generate(w)
@@ -837,6 +843,26 @@ def run_ours(args):
         "gpu_launches_isolated": 5 * min(max(K, 30), 200),
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_profile_launches(args, device):
+    """Isolated launches of every call for a profiler: one buffer set, each call
+    after a read-flush (so each starts on a clean L2 with its inputs in DRAM)."""
+    import torch
+    from combine_ep_layout_12_b200 import workloads as wl
+    w = wl.get(args.workload)
+    stream = torch.cuda.Stream(device)
+    wb = Workbench(w, wl.generate(w), device, stream, 1, 0)
+    p, d = wb.sets[0]
+    with torch.cuda.stream(stream):
+        for _ in range(args.profile_launches):
+            for name in ("layout", "dispatch", "layout_dispatch", "combine"):
+                wb.read_flush()
+                getattr(p, name)(d, stream)
+    stream.synchronize()
+    assert p.buf.check(stream) == 0, "device error bits set"
+    print("profile launches done: %s x %d" % (w.name, args.profile_launches), flush=True)
     return 0
 
 
