@@ -78,7 +78,9 @@ cudaError_t launch_int8(int U, dim3 grid, dim3 block, cudaStream_t stream, const
 //
 // Design (expert-major).  Each copy needs a whole fp32 smooth row, four times the
 // bytes of the int8 row it produces, so reading it per token (k rows per token)
-// makes the kernel bound by L2 reads of the table.  Instead a CTA takes one
+// makes the kernel bound by L2 reads of the table.  Instead the work is split by
+// expert.  Rows of up to 8192 elements take the column-owning kernel further
+// down; the row-wide kernel here takes any row length.  A CTA takes one
 // expert g and a share of its receive rows: it stages smooth[g] in shared memory
 // once, finds the source token of each of its rows through recv_src, and
 // quantizes the rows one at a time with all its threads.  Per-copy quantization
@@ -256,7 +258,241 @@ __global__ void __launch_bounds__(MAXT) dispatch_expert_major_kernel(ExpertArgs 
     }
 }
 
+// Column-owning form, for rows of up to 128 * 8 units of 8 elements (d <= 8192;
+// the row-wide kernel above takes longer rows).  A CTA of 128 threads (4 warps)
+// quantizes one receive row at a time, and thread i owns the same GP units
+// u = i + 128 m of every row, so the smooth values of its columns are loaded into
+// registers once per expert, and the per-row costs (the absmax reduction over four
+// warps, the scale division, the row bookkeeping) are spread over 8 GP elements per
+// thread.  x_fp32 is kept in registers between the absmax and the cast; the next
+// row's x is loaded while the current one is reduced.  The grid is one resident
+// wave: CTA b takes rows [N b / G, N (b + 1) / G) of the N routed rows in expert
+// order (row q of that order is copy q - expert_offset[g] of the expert g with
+// expert_offset[g] <= q < expert_offset[g + 1]), so every CTA has the same number
+// of rows and reloads the smooth row where its share crosses into the next expert.
+// Instruction savings that keep the bits: the absmax takes two elements per
+// three-operand maximum, and x_fp32 * s is formed two products per packed
+// multiply (each product rounded on its own; the add that follows is scalar, so no
+// multiply-add contraction can reach it).  A degenerate row takes s = 0, which
+// turns every finite x_fp32 into +-0 and so into the int8 code 0.
+constexpr int kColsThreads = 128;
+
+// (a.x * b.x, a.y * b.y), each product rounded to nearest even (one packed instruction)
+__device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {
+    unsigned long long ra, rb, rd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+    return d;
+}
+
+// max(a, |b|, |c|) in one three-operand maximum (NaN operands ignored, as fmaxf)
+__device__ __forceinline__ float fmax_abs2(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+    return r;
+}
+
+template <int GP, bool STATIC, bool EXACT>
+struct ColsRow {
+    const ExpertArgs& a;
+    const float4 (&sl)[GP];  // smooth[g][8u .. 8u + 3] of this thread's units
+    const float4 (&sh)[GP];  // smooth[g][8u + 4 .. 8u + 7]
+    int nu;
+    float (&red)[2][4];
+
+    // Quantizes the row (t, row) whose x is in cur; loads x of token t_next into nxt.
+    __device__ __forceinline__ void run(int t, long long row, int t_next, int& par, uint4 (&cur)[GP],
+                                        uint4 (&nxt)[GP]) const {
+        float f[GP][8];
+        float amax = 0.0f;
+#pragma unroll
+        for (int m = 0; m < GP; ++m) {
+            f[m][0] = __fmul_rn(bf16lo(cur[m].x), sl[m].x);
+            f[m][1] = __fmul_rn(bf16hi(cur[m].x), sl[m].y);
+            f[m][2] = __fmul_rn(bf16lo(cur[m].y), sl[m].z);
+            f[m][3] = __fmul_rn(bf16hi(cur[m].y), sl[m].w);
+            f[m][4] = __fmul_rn(bf16lo(cur[m].z), sh[m].x);
+            f[m][5] = __fmul_rn(bf16hi(cur[m].z), sh[m].y);
+            f[m][6] = __fmul_rn(bf16lo(cur[m].w), sh[m].z);
+            f[m][7] = __fmul_rn(bf16hi(cur[m].w), sh[m].w);
+            if (!STATIC) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) amax = fmax_abs2(amax, f[m][e], f[m][e + 1]);
+            }
+        }
+        const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(t_next < 0 ? 0 : t_next) * a.d);
+#pragma unroll
+        for (int m = 0; m < GP; ++m) {
+            const int u = threadIdx.x + m * kColsThreads;
+            nxt[m] = (t_next >= 0 && (EXACT || u < nu)) ? __ldg(xr + u) : make_uint4(0, 0, 0, 0);
+        }
+        float s = 1.0f;
+        bool degenerate = false;
+        if (!STATIC) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            if ((threadIdx.x & 31) == 0) red[par][threadIdx.x >> 5] = amax;
+            __syncthreads();
+            const float4 r4 = *reinterpret_cast<const float4*>(red[par]);
+            par ^= 1;
+            amax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
+            s = __fdiv_rn(127.0f, amax);
+            degenerate = (amax == 0.0f) || isinf(s);
+            if (degenerate) s = 0.0f;
+        }
+        if (t < 0) return;
+        uint2* out = reinterpret_cast<uint2*>(a.recv_x + row * a.d);
+#pragma unroll
+        for (int m = 0; m < GP; ++m) {
+            const int u = threadIdx.x + m * kColsThreads;
+            if (!EXACT && u >= nu) continue;
+            uint2 word;
+            if (STATIC) {
+                word.x = cvt_s8x4(f[m][0], f[m][1], f[m][2], f[m][3]);
+                word.y = cvt_s8x4(f[m][4], f[m][5], f[m][6], f[m][7]);
+            } else {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float2 p = fmul2_rn(make_float2(f[m][e], f[m][e + 1]), make_float2(s, s));
+                    v[e] = p.x;
+                    v[e + 1] = p.y;
+                }
+                word.x = cvt_s8x4_unclamped(v[0], v[1], v[2], v[3]);
+                word.y = cvt_s8x4_unclamped(v[4], v[5], v[6], v[7]);
+            }
+            out[u] = word;
+        }
+        if (!STATIC && threadIdx.x == 0) a.recv_scale[row] = degenerate ? 0.0f : __fdiv_rn(1.0f, s);
+    }
+};
+
+template <int GP, bool STATIC, bool EXACT>
+__global__ void __launch_bounds__(kColsThreads, 3) dispatch_expert_cols_kernel(ExpertArgs a) {
+    extern __shared__ int s_pre[];  // [P + 1]
+    __shared__ long long s_row[kColsThreads];
+    __shared__ int s_t[kColsThreads];
+    __shared__ __align__(16) float s_red[2][4];
+    constexpr int NT = kColsThreads;
+    const int nu = a.d >> 3;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_launch_dependents();
+    const long long N = min((long long)max(a.expert_offset[a.E], 0), a.rows);
+    long long q = N * blockIdx.x / gridDim.x;
+    const long long q1 = N * (blockIdx.x + 1) / gridDim.x;
+    int g = 0;
+    {
+        int lo = 0, hi = a.E - 1;  // the last expert whose rows start at or before q
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (a.expert_offset[mid] <= q) lo = mid; else hi = mid - 1;
+        }
+        g = lo;
+    }
+    float4 sl[GP], sh[GP];
+    const ColsRow<GP, STATIC, EXACT> body{a, sl, sh, nu, s_red};
+    int par = 0;
+    while (q < q1) {
+        while (g < a.E - 1 && a.expert_offset[g + 1] <= q) ++g;  // skip experts without rows
+        const long long off = a.expert_offset[g];
+        const long long end = min(q1, max(q + 1, (long long)a.expert_offset[g + 1]));
+        const float4* srow = reinterpret_cast<const float4*>(a.smooth + (size_t)g * a.d);
+#pragma unroll
+        for (int m = 0; m < GP; ++m) {
+            const int u = threadIdx.x + m * NT;
+            const bool in = EXACT || u < nu;
+            sl[m] = in ? __ldg(srow + 2 * u) : make_float4(0.f, 0.f, 0.f, 0.f);
+            sh[m] = in ? __ldg(srow + 2 * u + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (a.layout == 0 && warp == 0) {
+            // exclusive prefix over source ranks of this expert's row counts
+            int run = 0;
+            for (int r0 = 0; r0 < a.P; r0 += 32) {
+                const int r = r0 + lane;
+                const int c = r < a.P ? a.recv_count[(size_t)g * a.P + r] : 0;
+                int incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                if (r < a.P) s_pre[r] = run + incl - c;
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) s_pre[a.P] = run;
+        }
+        __syncthreads();
+        // copies of expert g that exist (an expert holds at most one copy per token)
+        const long long n = a.layout == 0 ? min((long long)s_pre[a.P], (long long)a.P * a.M) : end - off;
+        for (long long b0 = q; b0 < end; b0 += NT) {
+            const int nb = (int)min((long long)NT, end - b0);
+            if (threadIdx.x < nb) {
+                const long long i = b0 + threadIdx.x - off;
+                long long row = -1;
+                if (i >= 0 && i < n) {
+                    if (a.layout == 0) {
+                        int lo = 0, hi = a.P - 1;  // the last rank whose run starts at or before i
+                        while (lo < hi) {
+                            const int mid = (lo + hi + 1) >> 1;
+                            if (s_pre[mid] <= i) lo = mid; else hi = mid - 1;
+                        }
+                        row = (long long)g * a.P * a.M + (long long)lo * a.M + (i - s_pre[lo]);
+                    } else {
+                        row = b0 + threadIdx.x;
+                    }
+                }
+                const int t = (row >= 0 && row < a.rows) ? a.recv_src[row] : -1;
+                const bool ok = t >= 0 && t < a.B;
+                report_err(a.err, ok ? 0u : EP_ERRBIT_ROW_RANGE);
+                s_row[threadIdx.x] = row;
+                s_t[threadIdx.x] = ok ? t : -1;
+            }
+            __syncthreads();
+            uint4 xa[GP], xb[GP];
+            {
+                const int t0 = s_t[0];
+                const uint4* xr = reinterpret_cast<const uint4*>(a.x + (size_t)(t0 < 0 ? 0 : t0) * a.d);
+#pragma unroll
+                for (int m = 0; m < GP; ++m) {
+                    const int u = threadIdx.x + m * NT;
+                    xa[m] = (t0 >= 0 && (EXACT || u < nu)) ? __ldg(xr + u) : make_uint4(0, 0, 0, 0);
+                }
+            }
+            // two rows per iteration, so the current and the prefetched x swap roles
+            // without register copies
+            for (int j = 0; j < nb; j += 2) {
+                body.run(s_t[j], s_row[j], j + 1 < nb ? s_t[j + 1] : -1, par, xa, xb);
+                if (j + 1 < nb) body.run(s_t[j + 1], s_row[j + 1], j + 2 < nb ? s_t[j + 2] : -1, par, xb, xa);
+            }
+            __syncthreads();  // s_row / s_t (and s_pre) are rewritten next
+        }
+        q = end;
+        g = min(g + 1, a.E - 1);
+    }
+}
+
 using ExpertKernel = void (*)(ExpertArgs);
+
+ExpertKernel pick_cols_kernel(bool st, int GP, bool exact) {
+#define EP_COLS_K(G) \
+    (st ? (exact ? dispatch_expert_cols_kernel<G, true, true> : dispatch_expert_cols_kernel<G, true, false>) \
+        : (exact ? dispatch_expert_cols_kernel<G, false, true> : dispatch_expert_cols_kernel<G, false, false>))
+    switch (GP) {
+        case 1: return EP_COLS_K(1);
+        case 2: return EP_COLS_K(2);
+        case 3: return EP_COLS_K(3);
+        case 4: return EP_COLS_K(4);
+        case 5: return EP_COLS_K(5);
+        case 6: return EP_COLS_K(6);
+        case 7: return EP_COLS_K(7);
+        default: return EP_COLS_K(8);
+    }
+#undef EP_COLS_K
+}
 
 // GP units of 8 elements per thread, up to 256 threads (1024 for rows above 8192
 // elements), and whether NT * GP covers the row exactly.
@@ -305,9 +541,23 @@ int launch_dispatch_expert(const Shape& sh, const ep_buffer_ptrs& p, const uint1
     a.err = &reinterpret_cast<WsHeader*>(p.workspace)->err;
     a.rows = sh.rows;
     a.B = sh.B; a.d = sh.d; a.P = sh.P; a.M = sh.M; a.E = sh.E; a.layout = sh.layout;
+    const int nu = sh.d / 8;
+    if (nu <= kColsThreads * 8) {
+        const int GP = (nu + kColsThreads - 1) / kColsThreads;
+        const ExpertKernel kern = pick_cols_kernel(sh.quant_mode == 1, GP, GP * kColsThreads == nu);
+        const size_t smem = sizeof(int) * ((size_t)sh.P + 1);
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return EP_ERR_CUDA;
+        // one resident wave of CTAs, each with an equal share of the rows
+        const int occ = expert_occupancy(kern, kColsThreads, smem);
+        a.parts = 1;
+        const dim3 grid((unsigned)(num_sms() * occ));
+        const cudaError_t e = launch_pdl(kern, grid, dim3(kColsThreads), smem, stream, a);
+        return e == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+    }
     // units of 8 elements per thread: the smallest GP in {1, 2, 4} with at most 256
     // threads, else GP = 4 with up to 1024 threads (d <= 32768)
-    const int nu = sh.d / 8;
     int GP = 1;
     while (GP < 4 && (nu + GP - 1) / GP > 256) GP *= 2;
     int NT = (nu + GP - 1) / GP;

@@ -184,12 +184,27 @@ def test_expert_smooth(dev, name, kw):
 
 
 @pytest.mark.parametrize("qm", [1, 2])
-@pytest.mark.parametrize("d", [16, 272, 32768])
+@pytest.mark.parametrize("d", [16, 272, 4112, 8192, 8208, 32768])
 def test_expert_smooth_widths(dev, d, qm):
-    """Rows that do not tile the CTA (d = 16, 272) and the widest rows (1024 threads)."""
+    """Rows that do not tile the CTA (d = 16, 272, 4112), the widest rows with
+    columns owned per thread (8192), the first width past them (8208) and the
+    widest rows (1024 threads)."""
     w = wl.Workload("expert_d%d_q%d" % (d, qm), B=3 * 37, d=d, k=3, P=3, M=40, E=9, quant_mode=qm,
                     smooth="expert", seed=d)
     full_check(w, dev)
+
+
+@pytest.mark.parametrize("qm", [1, 2])
+def test_expert_smooth_degenerate_rows(dev, qm):
+    """Per-copy quantization of all-zero rows, rows whose 127/amax overflows and a
+    lone subnormal: q = 0 and scale 0 where the copy is degenerate."""
+    w = small("degenerate_expert", d=7168, smooth="expert", quant_mode=qm)
+    inp = wl.generate(w)
+    inp["x"][0] = 0
+    inp["x"][5] = 0x0080          # 2^-126 in every element: 127/amax overflows fp32
+    inp["x"][6, :] = 0
+    inp["x"][6, 3] = 0x8001       # a single negative subnormal
+    full_check(w, dev, inp=inp)
 
 
 def test_expert_smooth_dirty(dev):
