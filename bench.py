@@ -26,6 +26,7 @@ logical partitions of one GPU; nothing is exchanged between GPUs).
 import argparse
 import hashlib
 import json
+import re
 import os
 import statistics
 import sys
@@ -210,11 +211,25 @@ def trimmed_mean(xs, trim=0.1):
     return sum(xs) / len(xs)
 
 
-def source_hash(name):
+def code_text(src):
+    """C/C++/CUDA source without comments and with whitespace runs collapsed, so a
+    change to comments alone does not count as a change of the kernel."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
+def source_hash(name, read=None):
+    """Hash of the code of every source file a kernel is built from; read(rel) gives
+    a file's text (default: the working tree)."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES[name]:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        if read is None:
+            with open(os.path.join(ROOT, rel)) as f:
+                text = f.read()
+        else:
+            text = read(rel)
+        h.update(code_text(text).encode())
     return h.hexdigest()[:16]
 
 

@@ -94,10 +94,13 @@ __device__ __forceinline__ void combine_body(const CombineArgs& a, const Out& ou
     const int v_begin = c * span;
     const int v_end = min(nvec, v_begin + span);
 
-    // With self_rows the prologue only reads the routing (topk_idx, topk_weights),
-    // which was complete before the preceding kernels started, so it runs before
-    // griddepcontrol.wait and overlaps their tail; the expert outputs are read and
-    // y is written only after the wait.
+    // With self_rows the prologue reads the routing (topk_idx, topk_weights and the
+    // optional x_active_mask), which was complete before the preceding kernels
+    // started, and in the packed layout also expert_offset and recv_count, which
+    // ep_layout's counting kernel finished before the library's later kernels could
+    // start.  So it runs before griddepcontrol.wait and overlaps their tail; the
+    // expert outputs are read and y is written only after the wait.  (The public
+    // header states what a caller may therefore not launch in between.)
     __shared__ int s_rows[KMAX], s_g[KMAX], s_cnt[KMAX];
     // the weights were final before the preceding kernels started (as topk_idx):
     // their load is issued first so its latency overlaps the row lookup

@@ -27,6 +27,19 @@ def test_recorded_traffic_follows_the_source(tmp_path, monkeypatch):
     assert bench.recorded_traffic("other", "combine") is None
 
 
+def test_source_hash_ignores_comments_only():
+    """The recorded traffic stays valid across comment edits, not across code edits."""
+    base = "int f(int a) {\n  // twice a\n  return 2 * a; /* doubled */\n}\n"
+    comment_edit = "int f(int a) {\n  // two times a, reworded\n  return 2 * a;\n}\n"
+    code_edit = "int f(int a) {\n  // twice a\n  return 3 * a; /* doubled */\n}\n"
+    assert bench.code_text(base) == bench.code_text(comment_edit) == "int f(int a) { return 2 * a; }"
+    assert bench.code_text(base) != bench.code_text(code_edit)
+    files = {rel: base for rel in bench.KERNEL_SOURCES["combine"]}
+    h = bench.source_hash("combine", read=files.__getitem__)
+    assert h == bench.source_hash("combine", read={k: comment_edit for k in files}.__getitem__)
+    assert h != bench.source_hash("combine", read={k: code_edit for k in files}.__getitem__)
+
+
 def test_seeded_inputs_are_fixed():
     """The decode inputs every measurement and parity case uses do not drift."""
     inp = wl.generate(wl.get("decode"))
