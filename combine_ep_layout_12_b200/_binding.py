@@ -44,15 +44,17 @@ class ep_shard_table(ctypes.Structure):
     _fields_ = [("rank", ctypes.c_int32),
                 ("recv_x", ctypes.c_void_p * SHARD_MAX_RANKS),
                 ("recv_scale", ctypes.c_void_p * SHARD_MAX_RANKS),
-                ("recv_src", ctypes.c_void_p * SHARD_MAX_RANKS)]
+                ("recv_src", ctypes.c_void_p * SHARD_MAX_RANKS),
+                ("recv_count", ctypes.c_void_p * SHARD_MAX_RANKS)]
 
 
-def make_shard_table(rank, recv_x, recv_scale=None, recv_src=None):
+def make_shard_table(rank, recv_x, recv_scale=None, recv_src=None, recv_count=None):
     """ep_shard_table from per-rank device addresses (lists of ints; None entries or
     lists mean NULL)."""
     t = ep_shard_table()
     t.rank = int(rank)
-    for name, vals in (("recv_x", recv_x), ("recv_scale", recv_scale), ("recv_src", recv_src)):
+    for name, vals in (("recv_x", recv_x), ("recv_scale", recv_scale), ("recv_src", recv_src),
+                       ("recv_count", recv_count)):
         if vals is None:
             continue
         if len(vals) > SHARD_MAX_RANKS:
@@ -113,7 +115,7 @@ def _load(path):
     L.ep_layout_static_scratch.argtypes = [ctypes.POINTER(ep_config)] + [vp] * 8
     L.ep_shard_workspace_size.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ctypes.c_size_t)]
     L.ep_shard_layout.argtypes = [ctypes.POINTER(ep_config), ctypes.c_int32] + [vp] * 6
-    L.ep_shard_dispatch.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 6
+    L.ep_shard_dispatch.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 7
     L.ep_shard_combine.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 11
     L.ep_shard_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     for f in (L.ep_buffer_size, L.ep_buffer_create, L.ep_buffer_destroy, L.ep_layout,
@@ -203,9 +205,9 @@ def ep_shard_layout(cfg, rank, topk_idx, x_active_mask, dst_pos, send_count, wor
                                  send_count, workspace, stream), "ep_shard_layout")
 
 
-def ep_shard_dispatch(cfg, table, x, smooth_scale, dst_pos, token_scale, workspace, stream=0):
+def ep_shard_dispatch(cfg, table, x, smooth_scale, dst_pos, send_count, token_scale, workspace, stream=0):
     _check(lib().ep_shard_dispatch(ctypes.byref(cfg), ctypes.byref(table), x, smooth_scale, dst_pos,
-                                   token_scale, workspace, stream), "ep_shard_dispatch")
+                                   send_count, token_scale, workspace, stream), "ep_shard_dispatch")
 
 
 def ep_shard_combine(cfg, table, topk_idx, topk_weights, x_active_mask, dst_pos, ori_x, a1, a2, v, y,

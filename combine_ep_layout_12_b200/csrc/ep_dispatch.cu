@@ -43,12 +43,25 @@ __global__ void __launch_bounds__(256) dispatch_bf16_kernel(DispatchArgs a) {
     if (a.self_rows) pdl_wait();
 }
 
-// Multi-GPU form: rows read from dst_pos, stored into the owning rank's slab.
+// Multi-GPU form: rows read from dst_pos, stored into the owning rank's slab.  The
+// count exchange rides along: the threads of one CTA store this rank's send_count of
+// each expert g into column `rank` of the owner's recv_count (owner q = g / L, entry
+// [g - q L][rank]), plain stores to the owner's memory like the rows themselves.
+__device__ __forceinline__ void store_counts(const ShardTable& tab, int E) {
+    if (!tab.send_count) return;
+    for (int g = threadIdx.x; g < E; g += blockDim.x) {
+        const int q = g / tab.L;
+        int32_t* dst = tab.count[q];
+        if (dst) dst[(size_t)(g - q * tab.L) * tab.P + tab.rank] = tab.send_count[g];
+    }
+}
+
 template <int U, bool STATIC>
 __global__ void __launch_bounds__(256)
     dispatch_int8_shard_kernel(DispatchArgs a, const __grid_constant__ ShardTable tab) {
     pdl_wait();
     pdl_launch_dependents();
+    if (blockIdx.x == 0) store_counts(tab, a.E);
     dispatch_int8_body<U, STATIC>(a, blockIdx.x, ShardRows{tab});
 }
 
@@ -57,7 +70,15 @@ __global__ void __launch_bounds__(256)
     dispatch_bf16_shard_kernel(DispatchArgs a, const __grid_constant__ ShardTable tab) {
     pdl_wait();
     pdl_launch_dependents();
+    if (blockIdx.x == 0) store_counts(tab, a.E);
     dispatch_bf16_body<U>(a, blockIdx.x, ShardRows{tab});
+}
+
+// A rank without tokens still sends its (zero) counts.
+__global__ void __launch_bounds__(256) shard_counts_kernel(const __grid_constant__ ShardTable tab, int E) {
+    pdl_wait();
+    pdl_launch_dependents();
+    store_counts(tab, E);
 }
 
 template <bool STATIC>
@@ -621,7 +642,11 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
 
 int launch_shard_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
                           const float* smooth, const ShardTable& tab, cudaStream_t stream) {
-    if (s.B == 0) return EP_OK;
+    if (s.B == 0) {
+        if (!tab.send_count) return EP_OK;
+        return launch_pdl(shard_counts_kernel, dim3(1), dim3(256), 0, stream, tab, s.E) == cudaSuccess ? EP_OK
+                                                                                                  : EP_ERR_CUDA;
+    }
     DispatchArgs a = make_dispatch_args(s, p, x, smooth, nullptr, nullptr);
     a.self_rows = 0;
     int U = 0, NT = 0;

@@ -219,17 +219,24 @@ int shard_table(const ep_config* cfg, const ep_shard_table* tab, bool combine, e
         if (!combine && cfg->quant_mode == 2 && (!tab->recv_scale[q] || !aligned4(tab->recv_scale[q])))
             return EP_ERR_INVALID_ARG;
         if (!combine && tab->recv_src[q] && !aligned4(tab->recv_src[q])) return EP_ERR_INVALID_ARG;
+        if (!combine && tab->recv_count[q] && !aligned4(tab->recv_count[q])) return EP_ERR_INVALID_ARG;
         out->x[q] = tab->recv_x[q];
         out->scale[q] = combine ? nullptr : tab->recv_scale[q];
         out->src[q] = combine ? nullptr : tab->recv_src[q];
+        out->count[q] = combine ? nullptr : tab->recv_count[q];
     }
     for (int q = cfg->P; q < EP_SHARD_MAX_RANKS; ++q) {
         out->x[q] = nullptr;
         out->scale[q] = nullptr;
         out->src[q] = nullptr;
+        out->count[q] = nullptr;
     }
+    out->send_count = nullptr;
     out->slab_rows = (long long)(cfg->E / cfg->P) * cfg->P * cfg->M;
     out->token_base = tab->rank * (cfg->B / cfg->P);
+    out->rank = tab->rank;
+    out->P = cfg->P;
+    out->L = cfg->E / cfg->P;
     return EP_OK;
 }
 
@@ -269,8 +276,8 @@ int ep_shard_layout(const ep_config* cfg, int32_t rank, const int32_t* topk_idx,
 }
 
 int ep_shard_dispatch(const ep_config* cfg, const ep_shard_table* tab, const uint16_t* x,
-                      const float* smooth_scale, const int32_t* dst_pos, float* token_scale,
-                      void* workspace, ep_stream_t stream) {
+                      const float* smooth_scale, const int32_t* dst_pos, const int32_t* send_count,
+                      float* token_scale, void* workspace, ep_stream_t stream) {
     ep::Shape ls;
     ShardWs ws;
     int st = shard_local(cfg, &ls, &ws);
@@ -283,6 +290,8 @@ int ep_shard_dispatch(const ep_config* cfg, const ep_shard_table* tab, const uin
     if (ls.B > 0 && cfg->quant_mode == 2 && (!token_scale || !aligned4(token_scale))) return EP_ERR_INVALID_ARG;
     if (smooth_scale && (cfg->smooth_rows == 0 || cfg->quant_mode == 0 || !aligned16(smooth_scale)))
         return EP_ERR_INVALID_ARG;
+    if (send_count && !aligned4(send_count)) return EP_ERR_INVALID_ARG;
+    t.send_count = send_count;
     ep_buffer_ptrs p = {};
     p.dst_pos = const_cast<int32_t*>(dst_pos);
     p.token_scale = token_scale;

@@ -31,8 +31,11 @@ struct ShardTable {
     void* x[EP_SHARD_MAX_RANKS];        // recv_x slabs (dispatch) or expert-output slabs (combine)
     float* scale[EP_SHARD_MAX_RANKS];   // recv_scale slabs (dispatch, quant_mode 2)
     int32_t* src[EP_SHARD_MAX_RANKS];   // recv_src slabs (dispatch; may be null)
+    int32_t* count[EP_SHARD_MAX_RANKS]; // recv_count [L][P] of each rank (dispatch; may be null)
+    const int32_t* send_count;          // this rank's picks per expert [E] (dispatch; may be null)
     long long slab_rows;
     int token_base;                     // global index of this rank's first token
+    int rank, P, L;                     // this rank, the ranks, experts per rank
 };
 
 struct Shape {

@@ -9,21 +9,24 @@ one GPU.  One step of rank r:
 
   layout     ep_shard_layout: dst_pos [T, k] (global rows) and send_count [E]
   dispatch   ep_shard_dispatch: every routed copy stored straight into the owning
-             rank's slab (plain stores over NVLink), with its scale and source token
-  exchange   send_count[q*L:(q+1)*L] goes to rank q: one all-to-all; rank q gets
-             recv_count [L, P] (rows of each local expert from each source rank).
-             Issued after the dispatch, it also orders every rank's dispatch
-             before the experts read their slabs.
+             rank's slab (plain stores over NVLink), with its scale and source token;
+             the same kernel performs the count exchange: send_count[q*L:(q+1)*L]
+             stored into column r of rank q's recv_count [L, P] (rows of each local
+             expert from each source rank)
+  barrier    every rank's dispatch (rows and counts) is complete before any rank's
+             experts read their slab
   experts    the caller's function over this rank's slab (not part of this library)
   barrier    every rank's expert outputs are complete before any rank reads them
   combine    ep_shard_combine: each pick's expert output read from the owner's slab,
              reduced into y [T, d]
 
 Groups: LocalGroup runs the P logical ranks in one process on one GPU (P separate
-slab allocations; the exchange is a transpose and a barrier is stream order), and
-DistGroup runs one rank per process over torch.distributed (NCCL between GPUs, gloo
-on CPU for the host-side tests), mapping the peers' slabs through CUDA IPC.  torch
-supplies memory, streams and the collectives; every step of the data path runs in
+slab allocations; a barrier is stream order), and DistGroup runs one rank per
+process over torch.distributed (the barrier is a one-integer all-reduce, NCCL
+between GPUs, gloo on CPU for the host-side tests), mapping the peers' slabs
+through CUDA IPC.  exchange_count(s) are the same count exchange as a collective
+(all-to-all), for callers whose tables carry no recv_count addresses.  torch
+supplies memory, streams and the barriers; every step of the data path runs in
 libep's kernels.
 
 dbo(): the Wide-EP blog's dual-batch overlap, two micro-batches on two streams so
@@ -140,7 +143,7 @@ class Slab:
 
     def arrays(self):
         return {"recv_x": self.recv_x, "recv_scale": self.recv_scale, "recv_src": self.recv_src,
-                "expert_out": self.expert_out}
+                "recv_count": self.recv_count, "expert_out": self.expert_out}
 
 
 def _ptr(t):
@@ -171,7 +174,7 @@ class ShardRank:
         self.workspace = torch.zeros((nbytes,), dtype=torch.uint8, device=self.device)
         self.dispatch_table = abi.make_shard_table(
             rank, [_ptr(s["recv_x"]) for s in slabs], [_ptr(s.get("recv_scale")) for s in slabs],
-            [_ptr(s.get("recv_src")) for s in slabs])
+            [_ptr(s.get("recv_src")) for s in slabs], [_ptr(s.get("recv_count")) for s in slabs])
         self.combine_table = abi.make_shard_table(rank, [_ptr(s["expert_out"]) for s in slabs])
         self._keep = slabs  # the mapped peer tensors must outlive the tables
 
@@ -180,8 +183,11 @@ class ShardRank:
                             _ptr(self.send_count), _ptr(self.workspace), _stream(stream))
 
     def dispatch(self, x, smooth_scale=None, stream=None):
+        """Rows, scales and source tokens into the owners' slabs, and this rank's
+        send_count into column `rank` of every owner's recv_count."""
         abi.ep_shard_dispatch(self.cfg, self.dispatch_table, _ptr(x), _ptr(smooth_scale), _ptr(self.dst_pos),
-                              _ptr(self.token_scale), _ptr(self.workspace), _stream(stream))
+                              _ptr(self.send_count), _ptr(self.token_scale), _ptr(self.workspace),
+                              _stream(stream))
 
     def combine(self, topk_idx, topk_weights, x_active_mask=None, ori_x=None, a1=None, a2=None, v=None,
                 stream=None):
@@ -208,13 +214,17 @@ class LocalShards:
     def step(self, inputs, expert_fn=None, stream=None):
         """One step over per-rank inputs (a list over ranks of dicts with topk_idx,
         topk_weights, x and optional x_active_mask, smooth, a1, a2, v).  expert_fn(slab,
-        rank) fills slab.expert_out from the received rows (default: leave it as is)."""
+        rank) fills slab.expert_out from the received rows (default: leave it as is).
+        Everything, the count exchange and expert_fn included, runs on `stream`
+        (default: the current stream)."""
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+            return self._step(inputs, expert_fn, stream)
+
+    def _step(self, inputs, expert_fn, stream):
         for r, (rk, inp) in enumerate(zip(self.ranks, inputs)):
             rk.layout(inp["topk_idx"], inp.get("x_active_mask"), stream)
-            rk.dispatch(inp["x"], inp.get("smooth"), stream)
-        counts = self.group.exchange_counts([rk.send_count for rk in self.ranks])
-        for slab, c in zip(self.slabs, counts):
-            slab.recv_count.copy_(c)
+            rk.dispatch(inp["x"], inp.get("smooth"), stream)  # rows and counts into the owners' slabs
+        self.group.barrier()
         if expert_fn is not None:
             for r, slab in enumerate(self.slabs):
                 expert_fn(slab, r)
@@ -237,12 +247,17 @@ class DistShard:
         self.device = torch.device(device)
 
     def step(self, inp, expert_fn=None, stream=None):
-        """One step over this rank's inputs (dict as in LocalShards.step)."""
+        """One step over this rank's inputs (dict as in LocalShards.step).  The library
+        calls, the collectives and expert_fn all run on `stream` (default: the current
+        stream), so each collective is ordered after the kernels it depends on."""
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream()):
+            return self._step(inp, expert_fn, stream)
+
+    def _step(self, inp, expert_fn, stream):
         rk = self.rank
         rk.layout(inp["topk_idx"], inp.get("x_active_mask"), stream)
-        rk.dispatch(inp["x"], inp.get("smooth"), stream)
-        # the all-to-all also orders every rank's dispatch before this rank's experts
-        self.slab.recv_count.copy_(self.group.exchange_count(rk.send_count, self.cfg.P))
+        rk.dispatch(inp["x"], inp.get("smooth"), stream)  # rows and counts into the owners' slabs
+        self.group.barrier(self.device)  # every rank's dispatch is complete before the experts read
         if expert_fn is not None:
             expert_fn(self.slab, self.group.rank)
         self.group.barrier(self.device)  # every rank's expert outputs are complete

@@ -330,6 +330,11 @@ typedef struct {
                                                rows for ep_shard_combine */
     float* recv_scale[EP_SHARD_MAX_RANKS];  /* [P] recv_scale slabs [L*P*M] (quant_mode 2, dispatch) */
     int32_t* recv_src[EP_SHARD_MAX_RANKS];  /* [P] recv_src slabs [L*P*M] (dispatch); NULL = not written */
+    int32_t* recv_count[EP_SHARD_MAX_RANKS]; /* [P] rank q's recv_count [L][P] (dispatch, with a
+                                               send_count): the count exchange.  ep_shard_dispatch
+                                               stores column `rank` of every owner's array, entry
+                                               [l][rank] = this rank's picks of q's local expert l.
+                                               NULL = that rank's column is not written. */
 } ep_shard_table;
 
 /* Bytes of the device workspace of the ep_shard_* calls (one per process; the caller
@@ -345,10 +350,15 @@ EP_API int ep_shard_layout(const ep_config* cfg, int32_t rank, const int32_t* to
 
 /* Dispatch of rank tab->rank's tokens x (bf16 [T][d]) to the rows dst_pos of its
  * ep_shard_layout, into the slabs of `tab` (recv_x, recv_scale in quant_mode 2, recv_src
- * = rank*T + local token).  token_scale: fp32 [T] (quant_mode 2), else NULL. */
+ * = rank*T + local token).  token_scale: fp32 [T] (quant_mode 2), else NULL.
+ * send_count: the int32 [E] of the same ep_shard_layout, or NULL.  When given, the
+ * kernel also performs the count exchange: it stores send_count[q*L + l] into
+ * tab->recv_count[q][l*P + rank] for every rank q whose table entry is set (also when
+ * T = 0, so an owner never keeps a stale column).  Like the rows, those stores are
+ * ordered before another rank's reads by the caller's barrier after this call. */
 EP_API int ep_shard_dispatch(const ep_config* cfg, const ep_shard_table* tab, const uint16_t* x,
-                             const float* smooth_scale, const int32_t* dst_pos, float* token_scale,
-                             void* workspace, ep_stream_t stream);
+                             const float* smooth_scale, const int32_t* dst_pos, const int32_t* send_count,
+                             float* token_scale, void* workspace, ep_stream_t stream);
 
 /* Combine of rank tab->rank's tokens into y (bf16 [T][d]); tab->recv_x[q] are the bf16
  * expert-output slabs; other arguments as ep_combine, local to this rank. */

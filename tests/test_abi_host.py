@@ -196,20 +196,28 @@ def test_shard_calls_reject_bad_arguments_before_cuda():
     # a missing slab in the table
     holes = abi.make_shard_table(0, [fake] * 7 + [None], [fake] * 8, [fake] * 8)
     with pytest.raises(abi.EPError) as ei:
-        abi.ep_shard_dispatch(c, holes, fake, None, fake, fake, fake)
+        abi.ep_shard_dispatch(c, holes, fake, None, fake, None, fake, fake)
     assert ei.value.status == abi.EP_ERR_INVALID_ARG
     # a misaligned slab
     odd = abi.make_shard_table(0, [fake + 8] + [fake] * 7, [fake] * 8, [fake] * 8)
     with pytest.raises(abi.EPError) as ei:
-        abi.ep_shard_dispatch(c, odd, fake, None, fake, fake, fake)
+        abi.ep_shard_dispatch(c, odd, fake, None, fake, None, fake, fake)
     assert ei.value.status == abi.EP_ERR_INVALID_ARG
     # quant_mode 2 needs the scale slabs and token_scale
     no_scale = abi.make_shard_table(0, [fake] * 8, None, [fake] * 8)
     with pytest.raises(abi.EPError) as ei:
-        abi.ep_shard_dispatch(c, no_scale, fake, None, fake, fake, fake)
+        abi.ep_shard_dispatch(c, no_scale, fake, None, fake, None, fake, fake)
     assert ei.value.status == abi.EP_ERR_INVALID_ARG
     with pytest.raises(abi.EPError) as ei:
-        abi.ep_shard_dispatch(c, good, fake, None, fake, None, fake)
+        abi.ep_shard_dispatch(c, good, fake, None, fake, None, None, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    # the count exchange: a misaligned owner recv_count or send_count
+    odd_count = abi.make_shard_table(0, [fake] * 8, [fake] * 8, [fake] * 8, [fake] * 7 + [fake + 2])
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_dispatch(c, odd_count, fake, None, fake, fake, fake, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_dispatch(c, good, fake, None, fake, fake + 2, fake, fake)
     assert ei.value.status == abi.EP_ERR_INVALID_ARG
     # combine: y must be given and must not be ori_x
     with pytest.raises(abi.EPError) as ei:

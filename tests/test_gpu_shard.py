@@ -167,3 +167,22 @@ def test_shard_dbo_two_microbatches(dev):
     for got, want in ((ya, seq[0]), (yb, seq[1])):
         for g, s in zip(got, want):
             assert torch.equal(g, s)
+
+
+def test_shard_counts_with_empty_batch(dev):
+    """Ranks without tokens still perform the count exchange: every owner's recv_count
+    column is overwritten with zeros (no stale counts survive), and nothing else runs."""
+    w = wl.get("decode").with_(name="empty_shards", B=0, M=16, d=256)
+    sh = shard.LocalShards(w, dev)
+    for slab in sh.slabs:
+        slab.recv_count.fill_(-7)
+    k = w.k
+    inputs = [{"topk_idx": torch.empty((0, k), dtype=torch.int32, device=dev),
+               "topk_weights": torch.empty((0, k), dtype=torch.float32, device=dev),
+               "x": torch.empty((0, w.d), dtype=torch.bfloat16, device=dev)} for _ in range(w.P)]
+    ys = sh.step(inputs)
+    torch.cuda.synchronize()
+    for slab in sh.slabs:
+        assert int(slab.recv_count.abs().sum()) == 0
+    for rk, y in zip(sh.ranks, ys):
+        assert rk.check() == 0 and y.shape == (0, w.d)
