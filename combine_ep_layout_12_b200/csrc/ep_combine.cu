@@ -22,12 +22,6 @@
 namespace ep {
 namespace {
 
-#ifndef EP_COMBINE_PREFETCH
-#define EP_COMBINE_PREFETCH 0
-#endif
-// Column blocks (one per CTA pass over the row) prefetched into L2 ahead of the loads.
-constexpr int kCombinePrefetch = EP_COMBINE_PREFETCH;
-
 // Per-rank batches up to this size derive their rows from the routing (the scan of
 // the earlier tokens' ids stays within one load per thread).  At 256 tokens per
 // rank reading dst_pos was measured faster (90 against 102 us per combine at
@@ -148,22 +142,7 @@ __device__ __forceinline__ void combine_body(const CombineArgs& a, const Out& ou
     for (int j = 0; j < KMAX; ++j)
         if (j < a.k && s_ptr[j] != nullptr) live |= 1u << j;
 
-    // L2 prefetch, kCombinePrefetch column blocks ahead of the CTA's loads: thread j
-    // asks the copy engine for pick j's next block of row bytes, so more of the
-    // row is in flight than the loads' registers hold
-    const int NT = blockDim.x;
-    auto prefetch = [&](int blk) {
-        const int j = threadIdx.x;
-        const int v0 = v_begin + blk * NT;
-        if (kCombinePrefetch > 0 && j < KMAX && ((live >> j) & 1u) && v0 < v_end) {
-            const int nv = min(NT, v_end - v0);
-            bulk_prefetch_l2(s_ptr[j] + (size_t)v0 * 8, (uint32_t)nv * 16u);
-        }
-    };
-    for (int b = 0; b < kCombinePrefetch; ++b) prefetch(b);
-    int blk = 0;
-    for (int vcol = v_begin + threadIdx.x; vcol < v_end; vcol += blockDim.x, ++blk) {
-        if (kCombinePrefetch > 0) prefetch(blk + kCombinePrefetch);
+    for (int vcol = v_begin + threadIdx.x; vcol < v_end; vcol += blockDim.x) {
         const size_t col = (size_t)vcol * 8;
         uint4 raw[KMAX];
 #pragma unroll

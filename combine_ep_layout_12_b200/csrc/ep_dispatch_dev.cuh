@@ -11,15 +11,6 @@ namespace {
 
 constexpr int kSelfRowsMaxT = 256;
 
-#ifndef EP_DISPATCH_BULK
-#define EP_DISPATCH_BULK 0
-#endif
-// int8 rows of up to kBulkMaxD bytes: written once to shared memory and copied to
-// each receive row by the copy engine (cp.async.bulk shared -> global, no
-// multicast) instead of by k 16-byte stores per thread.
-constexpr bool kDispatchBulk = EP_DISPATCH_BULK != 0;
-constexpr int kBulkMaxD = 8192;
-
 struct DispatchArgs {
     const uint16_t* x;       // [B][d] bf16
     const float* smooth;     // [d] or null
@@ -48,7 +39,6 @@ struct DispatchArgs {
 //  lookup with a computed rank index reads the parameter bank, not a local copy.
 //  recv_src is written here too (the sender is the only one that knows the token).
 struct LocalRows {
-    static constexpr bool kBulk = true;  // bulk copies only into this GPU's own memory
     __device__ __forceinline__ char* x(const DispatchArgs& a, int row, size_t row_bytes) const {
         return reinterpret_cast<char*>(a.recv_x) + (size_t)row * row_bytes;
     }
@@ -57,7 +47,6 @@ struct LocalRows {
 };
 
 struct ShardRows {
-    static constexpr bool kBulk = false;
     const ShardTable& tab;
     __device__ __forceinline__ char* x(const DispatchArgs&, int row, size_t row_bytes) const {
         const int q = (int)(row / tab.slab_rows);
@@ -168,8 +157,6 @@ template <int U, bool STATIC, class Rows = LocalRows>
 __device__ __forceinline__ void dispatch_int8_body(const DispatchArgs& a, int t, const Rows& rows = Rows()) {
     __shared__ int s_rows[kMaxK];
     __shared__ char* s_dst[kMaxK];
-    __shared__ __align__(128) uint8_t s_row[kDispatchBulk && Rows::kBulk ? kBulkMaxD : 16];
-    const bool bulk = kDispatchBulk && Rows::kBulk && a.d <= kBulkMaxD;
     __shared__ float s_red[32];
     const int nunits = a.d >> 4;
     const int NT = blockDim.x;
@@ -265,27 +252,9 @@ __device__ __forceinline__ void dispatch_int8_body(const DispatchArgs& a, int t,
                            cvt_s8x4_unclamped(f[8], f[9], f[10], f[11]),
                            cvt_s8x4_unclamped(f[12], f[13], f[14], f[15]));
         if (degenerate) v = make_uint4(0, 0, 0, 0);
-        if (bulk) {
-            *reinterpret_cast<uint4*>(s_row + 16 * u) = v;
-        } else {
-            for (int j = 0; j < a.k; ++j) {
-                char* dst = s_dst[j];
-                if (dst) st_v4(dst + 16 * u, v);
-            }
-        }
-    }
-    if (bulk) {
-        // the whole int8 row is in shared memory: thread j copies it to pick j's row
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        __syncthreads();
-        if (threadIdx.x < a.k && s_dst[threadIdx.x]) {
-            const uint32_t saddr = (uint32_t)__cvta_generic_to_shared(s_row);
-            asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(s_dst[threadIdx.x]),
-                         "r"(saddr), "r"((uint32_t)a.d)
-                         : "memory");
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            // the staged row must stay in place until the copy has read it
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        for (int j = 0; j < a.k; ++j) {
+            char* dst = s_dst[j];
+            if (dst) st_v4(dst + 16 * u, v);
         }
     }
     if (STATIC) return;

@@ -181,12 +181,6 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                  "r"(v.z), "r"(v.w));
 }
 
-// Ask the copy engine to bring [p, p + bytes) into L2 (no data returned to the SM;
-// p and bytes 16-byte aligned).
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes));
-}
-
 // bf16 bits <-> fp32: a bf16 is the high half of a binary32.
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
