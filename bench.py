@@ -67,6 +67,8 @@ def parse_args(argv=None):
     p.add_argument("--sweep", default=None,
                    help="comma-separated workloads or 'all': per-workload table instead of the JSON line")
     p.add_argument("--sweep-out", default=None, help="where --sweep writes its JSON document")
+    p.add_argument("--shard", action="store_true",
+                   help="time the multi-GPU form on this GPU (P slabs, two micro-batches, dual-batch overlap)")
     p.add_argument("--profile-launches", type=int, default=0, metavar="N",
                    help="for profiler captures: build --workload with one buffer set and run N times each "
                         "of ep_layout, ep_dispatch, ep_layout_dispatch and ep_combine, each after an L2 "
@@ -632,6 +634,8 @@ def run_ours(args):
         return run_sweep(args, device)
     if args.profile_launches:
         return run_profile_launches(args, device)
+    if args.shard:
+        return run_shard(args, device)
 
     w = wl.get(args.workload)
     inp = wl.generate(w)
@@ -879,6 +883,99 @@ def run_profile_launches(args, device):
     assert p.buf.check(stream) == 0, "device error bits set"
     print("profile launches done: %s x %d" % (w.name, args.profile_launches), flush=True)
     return 0
+
+
+def run_shard(args, device):
+    """The multi-GPU form on one GPU: the P logical ranks of --workload in one process,
+    each with its own slab allocation, reached through the pointer tables a multi-GPU
+    run fills with mapped peer slabs; the ranks' kernels in turn on one stream, then on
+    a stream per rank (as P GPUs run them).  Times, as CUDA graphs replayed K times:
+    - one step of one micro-batch: every rank's layout, dispatch (with the in-kernel
+      count exchange) and combine;
+    - two micro-batches (different routing and tokens) one after the other;
+    - the same two with the dual-batch overlap (shard.dbo, two streams).
+    The expert outputs are filled once and not recomputed (the experts are not part
+    of the path).  Prints one JSON line per arrangement; --sweep-out also writes them
+    to a file."""
+    import torch
+    from combine_ep_layout_12_b200 import workloads as wl
+    wa = wl.get(args.workload)
+    wb_ = wa.with_(name=wa.name + "_b", seed=wa.seed + 1)
+    stream = torch.cuda.Stream(device)
+    side = torch.cuda.Stream(device)
+    lines = []
+    for rank_streams in (False, True):
+        lines.append(_shard_times(args, device, wa, wb_, stream, side, rank_streams))
+        print(json.dumps(lines[-1]), flush=True)
+        torch.cuda.empty_cache()
+    if args.sweep_out:
+        with open(args.sweep_out, "w") as f:
+            json.dump(lines, f, indent=1)
+    return 0
+
+
+def _shard_times(args, device, wa, wb_, stream, side, rank_streams):
+    """The three graph timings of run_shard for one arrangement of the ranks."""
+    import torch
+    from combine_ep_layout_12_b200 import metrics, runner, shard
+    from combine_ep_layout_12_b200 import workloads as wl
+    shards, inputs, nbytes = [], [], 0.0
+    for w in (wa, wb_):
+        inp = wl.generate(w)
+        n_routed, b_sp = metrics.routing_counts(w, inp["topk_idx"], active=inp.get("active"))
+        kb = metrics.kernel_bytes(w, n_routed, b_sp, smooth=inp.get("smooth") is not None,
+                                  masked=inp.get("active") is not None)
+        nbytes += float(sum(kb.values()))
+        sh = shard.LocalShards(w, device, rank_streams=rank_streams)
+        for slab in sh.slabs:
+            slab.expert_out.normal_()
+        shards.append(sh)
+        inputs.append(shard.split_inputs(w, runner.to_device(inp, device)))
+    sa, sb = shards
+    ra, rb = inputs
+    with torch.cuda.stream(stream):
+        sa.step(ra, None, stream)
+        sb.step(rb, None, stream)
+    stream.synchronize()
+    for sh in shards:
+        for rk in sh.ranks:
+            assert rk.check() == 0, "device error bits set"
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        return g
+
+    graphs = {"one_step": capture(lambda: sa.step(ra, None, stream)),
+              "two_sequential": capture(lambda: (sa.step(ra, None, stream), sb.step(rb, None, stream))),
+              "two_dbo": capture(lambda: shard.dbo(sa, sb, ra, rb, None, (stream, side)))}
+    K = max(3, min(args.steps, 200))
+    res = {}
+    for name, g in graphs.items():
+        for _ in range(max(3, args.warmup)):
+            g.replay()
+        torch.cuda.synchronize(device)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(K):
+                g.replay()
+        t1.record(stream)
+        t1.synchronize()
+        res[name] = 1e3 * t0.elapsed_time(t1) / K
+    for sh in shards:
+        for rk in sh.ranks:
+            assert rk.check() == 0, "device error bits set"
+    one = res["one_step"]
+    line = {"mode": "shard, one GPU", "ranks": "concurrent, one stream per rank" if rank_streams else "in turn, one stream",
+            "workload": wa.name, "P": wa.P, "T": wa.T, "steps": K,
+            "one_step_us": one, "one_step_gbs": nbytes / 2 / (one * 1e-6) / 1e9,
+            "two_sequential_us": res["two_sequential"], "two_dbo_us": res["two_dbo"],
+            "dbo_speedup": res["two_sequential"] / res["two_dbo"]}
+    del graphs
+    return line
 
 
 def fit_latency_bandwidth(points):

@@ -66,6 +66,23 @@ def send_slices(cfg, send_count):
     return send_count.reshape(cfg.P, local_experts(cfg))
 
 
+def split_inputs(cfg, inputs):
+    """Device inputs of the whole batch (dict: topk_idx [B, k], topk_weights, x, and the
+    optional smooth, a1, a2, v, active) -> a list over ranks of the dicts that
+    LocalShards.step takes: rank r's tokens r*T .. r*T+T-1, the shared tables as they are."""
+    T = cfg.B // cfg.P
+    out = []
+    for r in range(cfg.P):
+        sl = slice(r * T, (r + 1) * T)
+        d = {"topk_idx": inputs["topk_idx"][sl].contiguous(), "topk_weights": inputs["topk_weights"][sl].contiguous(),
+             "x": inputs["x"][sl].contiguous(), "smooth": inputs.get("smooth"), "a1": inputs.get("a1"),
+             "a2": inputs.get("a2"), "v": inputs.get("v")}
+        if inputs.get("active") is not None:
+            d["x_active_mask"] = inputs["active"][sl].contiguous()
+        out.append(d)
+    return out
+
+
 # ----------------------------------------------------------------------------- groups
 
 
@@ -202,14 +219,35 @@ class ShardRank:
 
 class LocalShards:
     """All P logical ranks of one micro-batch in one process on one GPU: P separate
-    slab allocations and one ShardRank per rank."""
+    slab allocations and one ShardRank per rank.  With rank_streams each rank's
+    kernels go to a stream of its own, forked from and joined back to the step's
+    stream at the two points where ranks meet (after every dispatch, after every
+    combine), as P GPUs would run them; otherwise the ranks run in turn."""
 
-    def __init__(self, cfg, device):
+    def __init__(self, cfg, device, rank_streams=False):
         self.cfg = cfg
         self.group = LocalGroup(cfg.P)
         self.slabs = [Slab(cfg, device) for _ in range(cfg.P)]
         tabs = [s.arrays() for s in self.slabs]
         self.ranks = [ShardRank(cfg, r, tabs, device) for r in range(cfg.P)]
+        self.streams = [torch.cuda.Stream(device) for _ in range(cfg.P)] if rank_streams else None
+
+    def _per_rank(self, main, fn):
+        """fn(r, stream) for every rank: on `main` in turn, or forked onto the ranks'
+        streams and joined back to `main`."""
+        if self.streams is None:
+            return [fn(r, main) for r in range(self.cfg.P)]
+        start = torch.cuda.Event()
+        start.record(main)
+        out = []
+        for r, st in enumerate(self.streams):
+            st.wait_event(start)
+            with torch.cuda.stream(st):
+                out.append(fn(r, st))
+            done = torch.cuda.Event()
+            done.record(st)
+            main.wait_event(done)
+        return out
 
     def step(self, inputs, expert_fn=None, stream=None):
         """One step over per-rank inputs (a list over ranks of dicts with topk_idx,
@@ -221,17 +259,25 @@ class LocalShards:
             return self._step(inputs, expert_fn, stream)
 
     def _step(self, inputs, expert_fn, stream):
-        for r, (rk, inp) in enumerate(zip(self.ranks, inputs)):
-            rk.layout(inp["topk_idx"], inp.get("x_active_mask"), stream)
-            rk.dispatch(inp["x"], inp.get("smooth"), stream)  # rows and counts into the owners' slabs
+        main = torch.cuda.current_stream()
+
+        def send(r, st):
+            rk, inp = self.ranks[r], inputs[r]
+            rk.layout(inp["topk_idx"], inp.get("x_active_mask"), st)
+            rk.dispatch(inp["x"], inp.get("smooth"), st)  # rows and counts into the owners' slabs
+
+        def receive(r, st):
+            rk, inp = self.ranks[r], inputs[r]
+            return rk.combine(inp["topk_idx"], inp["topk_weights"], inp.get("x_active_mask"), inp["x"],
+                              inp.get("a1"), inp.get("a2"), inp.get("v"), st)
+
+        self._per_rank(main, send)
         self.group.barrier()
         if expert_fn is not None:
             for r, slab in enumerate(self.slabs):
                 expert_fn(slab, r)
         self.group.barrier()
-        return [rk.combine(inp["topk_idx"], inp["topk_weights"], inp.get("x_active_mask"), inp["x"],
-                           inp.get("a1"), inp.get("a2"), inp.get("v"), stream)
-                for rk, inp in zip(self.ranks, inputs)]
+        return self._per_rank(main, receive)
 
 
 class DistShard:

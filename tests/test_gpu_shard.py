@@ -40,17 +40,7 @@ CASES = {
 
 
 def _per_rank(w, dev_inp):
-    T = w.B // w.P
-    out = []
-    for r in range(w.P):
-        sl = slice(r * T, (r + 1) * T)
-        d = {"topk_idx": dev_inp["topk_idx"][sl].contiguous(), "topk_weights": dev_inp["topk_weights"][sl].contiguous(),
-             "x": dev_inp["x"][sl].contiguous(), "smooth": dev_inp.get("smooth"), "a1": dev_inp.get("a1"),
-             "a2": dev_inp.get("a2"), "v": dev_inp.get("v")}
-        if dev_inp.get("active") is not None:
-            d["x_active_mask"] = dev_inp["active"][sl].contiguous()
-        out.append(d)
-    return out
+    return shard.split_inputs(w, dev_inp)
 
 
 def _expert_rows(w, ref, seed_offset=0):
@@ -140,6 +130,13 @@ def test_shard_step_matches_oracle(dev, name):
     if gp.need_bytes(w, True) > gp.free_bytes() - (4 << 30):
         pytest.skip("needs %.1f GB" % (gp.need_bytes(w, True) / 1e9))
     _check(w, *_run(w, dev))
+
+
+def test_shard_rank_streams(dev):
+    """Each rank's kernels on a stream of its own (as P GPUs run them), joined where
+    ranks meet: the same results as the ranks in turn."""
+    w = CASES["skewed"]
+    _check(w, *_run(w, dev, shards=shard.LocalShards(w, dev, rank_streams=True)))
 
 
 def test_shard_dbo_two_microbatches(dev):
