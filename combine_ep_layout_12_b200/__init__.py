@@ -20,7 +20,8 @@ Usage (one decode step of 8 logical ranks x 128 tokens, DeepSeek-V3 shape):
     y = buf.combine(expert_out, topk_idx, topk_weights, ori_x=x)
 
 Across GPUs (one process per GPU, each holding one logical rank's tokens and its
-receive slab): see shard.py (ep_shard_layout / ep_shard_dispatch / ep_shard_combine).
+receive slab): see shard.py (ep_shard_layout / ep_shard_dispatch / ep_shard_layout_dispatch /
+ep_shard_combine).
 
 Options: quant_mode 0 (bf16) / 1 (static int8) / 2 (dynamic int8); smooth_rows
 = E for a per-expert [E, d] smooth scale; layout=1 for rows packed per expert
@@ -34,13 +35,13 @@ from . import _binding as abi
 from ._binding import (EPError, ep_buffer_check, ep_buffer_create, ep_buffer_destroy,
                        ep_buffer_size, ep_combine, ep_dispatch, ep_layout, ep_layout_dispatch,
                        ep_layout_static_scratch, ep_shard_check, ep_shard_combine, ep_shard_dispatch,
-                       ep_shard_layout, ep_shard_workspace_size, ep_status_str, make_config,
+                       ep_shard_layout, ep_shard_layout_dispatch, ep_shard_workspace_size, ep_status_str, make_config,
                        make_shard_table)
 
 __all__ = ["EPBuffer", "EPError", "abi", "ep_buffer_check", "ep_buffer_create",
            "ep_buffer_destroy", "ep_buffer_size", "ep_combine", "ep_dispatch", "ep_layout",
            "ep_layout_dispatch", "ep_layout_static_scratch", "ep_shard_check", "ep_shard_combine",
-           "ep_shard_dispatch", "ep_shard_layout", "ep_shard_workspace_size", "ep_status_str",
+           "ep_shard_dispatch", "ep_shard_layout", "ep_shard_layout_dispatch", "ep_shard_workspace_size", "ep_status_str",
            "make_config", "make_shard_table"]
 
 

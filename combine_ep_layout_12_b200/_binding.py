@@ -116,12 +116,13 @@ def _load(path):
     L.ep_shard_workspace_size.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ctypes.c_size_t)]
     L.ep_shard_layout.argtypes = [ctypes.POINTER(ep_config), ctypes.c_int32] + [vp] * 6
     L.ep_shard_dispatch.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 7
+    L.ep_shard_layout_dispatch.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 9
     L.ep_shard_combine.argtypes = [ctypes.POINTER(ep_config), ctypes.POINTER(ep_shard_table)] + [vp] * 11
     L.ep_shard_check.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     for f in (L.ep_buffer_size, L.ep_buffer_create, L.ep_buffer_destroy, L.ep_layout,
               L.ep_dispatch, L.ep_layout_dispatch, L.ep_combine, L.ep_buffer_check,
               L.ep_layout_static_scratch, L.ep_shard_workspace_size, L.ep_shard_layout,
-              L.ep_shard_dispatch, L.ep_shard_combine, L.ep_shard_check):
+              L.ep_shard_dispatch, L.ep_shard_layout_dispatch, L.ep_shard_combine, L.ep_shard_check):
         f.restype = i
     L.ep_status_str.argtypes = [i]
     L.ep_status_str.restype = ctypes.c_char_p
@@ -208,6 +209,13 @@ def ep_shard_layout(cfg, rank, topk_idx, x_active_mask, dst_pos, send_count, wor
 def ep_shard_dispatch(cfg, table, x, smooth_scale, dst_pos, send_count, token_scale, workspace, stream=0):
     _check(lib().ep_shard_dispatch(ctypes.byref(cfg), ctypes.byref(table), x, smooth_scale, dst_pos,
                                    send_count, token_scale, workspace, stream), "ep_shard_dispatch")
+
+
+def ep_shard_layout_dispatch(cfg, table, topk_idx, x_active_mask, x, smooth_scale, dst_pos, send_count,
+                             token_scale, workspace, stream=0):
+    _check(lib().ep_shard_layout_dispatch(ctypes.byref(cfg), ctypes.byref(table), topk_idx, x_active_mask, x,
+                                          smooth_scale, dst_pos, send_count, token_scale, workspace, stream),
+           "ep_shard_layout_dispatch")
 
 
 def ep_shard_combine(cfg, table, topk_idx, topk_weights, x_active_mask, dst_pos, ori_x, a1, a2, v, y,

@@ -22,6 +22,7 @@ struct DispatchArgs {
     const int32_t* expert_offset;  // packed rows with self_rows: the layout's counts
     const int32_t* recv_count;
     int T, P, M, E;
+    int gstride, rbase;      // self_rows: row of (g, rank r, slot) = g * gstride + r * M + rbase + slot
     void* recv_x;            // [rows][d] int8 or bf16
     float* recv_scale;       // [rows]
     float* token_scale;      // [B]
@@ -84,7 +85,7 @@ __device__ __forceinline__ void compute_rows(const DispatchArgs& a, int t, int* 
                                              int* s_cnt) {
     __shared__ uint16_t s_tab[kMaxE];
     routing_rows(a.topk_idx, a.active, t, a.k, a.E, a.T, a.P, a.M, s_rows, s_g, s_cnt, s_tab,
-                 a.expert_offset, a.recv_count);
+                 a.expert_offset, a.recv_count, a.gstride, a.rbase);
 }
 
 // Receive rows of token t into shared memory; out-of-range rows are skipped and flagged.
@@ -321,6 +322,8 @@ inline DispatchArgs make_dispatch_args(const Shape& s, const ep_buffer_ptrs& p, 
     a.P = s.P;
     a.M = s.M;
     a.E = s.E;
+    a.gstride = s.P * s.M;
+    a.rbase = 0;
     return a;
 }
 

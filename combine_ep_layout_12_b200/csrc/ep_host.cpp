@@ -299,6 +299,36 @@ int ep_shard_dispatch(const ep_config* cfg, const ep_shard_table* tab, const uin
     return ep::launch_shard_dispatch(ls, p, x, smooth_scale, t, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int ep_shard_layout_dispatch(const ep_config* cfg, const ep_shard_table* tab, const int32_t* topk_idx,
+                             const uint8_t* x_active_mask, const uint16_t* x, const float* smooth_scale,
+                             int32_t* dst_pos, int32_t* send_count, float* token_scale, void* workspace,
+                             ep_stream_t stream) {
+    ep::Shape ls;
+    ShardWs ws;
+    int st = shard_local(cfg, &ls, &ws);
+    if (st != EP_OK) return st;
+    ep::ShardTable t;
+    st = shard_table(cfg, tab, false, &t);
+    if (st != EP_OK) return st;
+    if (!workspace || !aligned16(workspace) || !send_count || !aligned4(send_count)) return EP_ERR_INVALID_ARG;
+    if (ls.B > 0 && (!topk_idx || !aligned4(topk_idx) || !dst_pos || !aligned4(dst_pos) || !x || !aligned16(x)))
+        return EP_ERR_INVALID_ARG;
+    if (ls.B > 0 && cfg->quant_mode == 2 && (!token_scale || !aligned4(token_scale))) return EP_ERR_INVALID_ARG;
+    if (smooth_scale && (cfg->smooth_rows == 0 || cfg->quant_mode == 0 || !aligned16(smooth_scale)))
+        return EP_ERR_INVALID_ARG;
+    ep_buffer_ptrs p = {};
+    char* w = static_cast<char*>(workspace);
+    p.expert_count = reinterpret_cast<int32_t*>(w + ws.count_off);
+    p.expert_offset = reinterpret_cast<int32_t*>(w + ws.offset_off);
+    p.recv_count = send_count;  // [E][1]: this rank's column
+    p.dst_pos = dst_pos;
+    p.recv_src = nullptr;       // written by the dispatch, into the owners' slabs
+    p.token_scale = token_scale;
+    p.workspace = workspace;
+    return ep::launch_shard_layout_dispatch(ls, p, topk_idx, x_active_mask, x, smooth_scale, t, cfg->P * cfg->M,
+                                            tab->rank * cfg->M, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int ep_shard_combine(const ep_config* cfg, const ep_shard_table* tab, const int32_t* topk_idx,
                      const float* topk_weights, const uint8_t* x_active_mask, const int32_t* dst_pos,
                      const uint16_t* ori_x, const uint16_t* a1, const uint16_t* a2, const uint16_t* v,

@@ -99,6 +99,12 @@ int launch_combine(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* expe
 // view: B = T tokens of this rank, rows = the global E * P * M.
 int launch_shard_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
                           const float* smooth, const ShardTable& tab, cudaStream_t stream);
+// Layout and dispatch of one rank (s: P = 1, global rows via gstride and rbase) with
+// the count exchange, in one grid when T <= 128 and k <= 8; p.recv_count is the
+// rank's send_count [E].
+int launch_shard_layout_dispatch(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
+                                 const uint8_t* active, const uint16_t* x, const float* smooth,
+                                 const ShardTable& tab, int gstride, int rbase, cudaStream_t stream);
 int launch_shard_combine(const Shape& s, const ep_buffer_ptrs& p, const int32_t* topk_idx,
                          const float* topk_weights, const uint8_t* active, const uint16_t* ori_x,
                          const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
@@ -237,7 +243,7 @@ __device__ __forceinline__ void report_err(unsigned* err_word, unsigned bits) {
 __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* active, int t, int k,
                                     int E, int T, int P, int M, int* s_rows, int* s_g, int* s_cnt,
                                     uint16_t* tab, const int32_t* expert_offset = nullptr,
-                                    const int32_t* recv_count = nullptr) {
+                                    const int32_t* recv_count = nullptr, int gstride = -1, int rbase = 0) {
     uint32_t* tw = reinterpret_cast<uint32_t*>(tab);
     for (int i = threadIdx.x; i < (E + 1) / 2; i += blockDim.x) tw[i] = 0u;
     if (threadIdx.x < k) {
@@ -293,7 +299,9 @@ __device__ inline void routing_rows(const int32_t* topk_idx, const uint8_t* acti
     if (threadIdx.x < k) {
         const int g = s_g[threadIdx.x];
         int row = -1;
-        if (g >= 0) row = expert_offset ? s_cnt[threadIdx.x] : g * P * M + r * M + s_cnt[threadIdx.x];
+        if (g >= 0)
+            row = expert_offset ? s_cnt[threadIdx.x]
+                                : g * (gstride < 0 ? P * M : gstride) + r * M + rbase + s_cnt[threadIdx.x];
         s_rows[threadIdx.x] = row;
     }
 }

@@ -139,9 +139,12 @@ __device__ __forceinline__ unsigned classify_ids(const int* ids, int k, int E, i
 //    sum of its ranks' chunk popcounts per expert is recv_count.
 // Each warp reads only its own tokens' ids, and both halves use order-independent
 // shared-memory atomics, so the result is deterministic.
+// shard (multi-GPU form, one rank laid out as P = 1): when given, the slot CTA also
+// stores each expert's count into column shard->rank of the owning rank's recv_count,
+// which is the count exchange of ep_shard_layout_dispatch.
 template <int KM>
 __device__ __forceinline__ void layout_small_body(const LayoutArgs& a, int cpr, int cta,
-                                                  unsigned* smem) {
+                                                  unsigned* smem, const ShardTable* shard = nullptr) {
     const int E = a.E, k = a.k, P = a.P;
     const bool vec4 = (k % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.topk_idx) & 15) == 0);
     unsigned err = 0;
@@ -233,6 +236,10 @@ __device__ __forceinline__ void layout_small_body(const LayoutArgs& a, int cpr, 
         int n = 0;
         for (int cc = 0; cc < cpr; ++cc) n += __popc(mask[(size_t)(lrr * cpr + cc) * E + g]);
         a.recv_count[(size_t)g * P + rr] = n;
+        if (shard) {
+            const int q = g / shard->L;
+            if (shard->count[q]) shard->count[q][(size_t)(g - q * shard->L) * shard->P + shard->rank] = n;
+        }
     }
     // errors of the chunk's own tokens only (the count CTA reports the same bits)
     report_err(&a.ws->err, err);

@@ -13,6 +13,8 @@ one GPU.  One step of rank r:
              the same kernel performs the count exchange: send_count[q*L:(q+1)*L]
              stored into column r of rank q's recv_count [L, P] (rows of each local
              expert from each source rank)
+             (ep_shard_layout_dispatch does layout and dispatch as one call, one grid
+             for T <= 128, the way ep_layout_dispatch does on one GPU)
   barrier    every rank's dispatch (rows and counts) is complete before any rank's
              experts read their slab
   experts    the caller's function over this rank's slab (not part of this library)
@@ -206,6 +208,13 @@ class ShardRank:
                               _ptr(self.send_count), _ptr(self.token_scale), _ptr(self.workspace),
                               _stream(stream))
 
+    def layout_dispatch(self, topk_idx, x, x_active_mask=None, smooth_scale=None, stream=None):
+        """layout and dispatch (with the count exchange) as one call: one grid when
+        T <= 128 and k <= 8."""
+        abi.ep_shard_layout_dispatch(self.cfg, self.dispatch_table, _ptr(topk_idx), _ptr(x_active_mask), _ptr(x),
+                                     _ptr(smooth_scale), _ptr(self.dst_pos), _ptr(self.send_count),
+                                     _ptr(self.token_scale), _ptr(self.workspace), _stream(stream))
+
     def combine(self, topk_idx, topk_weights, x_active_mask=None, ori_x=None, a1=None, a2=None, v=None,
                 stream=None):
         abi.ep_shard_combine(self.cfg, self.combine_table, _ptr(topk_idx), _ptr(topk_weights),
@@ -224,8 +233,9 @@ class LocalShards:
     stream at the two points where ranks meet (after every dispatch, after every
     combine), as P GPUs would run them; otherwise the ranks run in turn."""
 
-    def __init__(self, cfg, device, rank_streams=False):
+    def __init__(self, cfg, device, rank_streams=False, fused=True):
         self.cfg = cfg
+        self.fused = fused  # layout and dispatch as one call (ep_shard_layout_dispatch)
         self.group = LocalGroup(cfg.P)
         self.slabs = [Slab(cfg, device) for _ in range(cfg.P)]
         tabs = [s.arrays() for s in self.slabs]
@@ -261,10 +271,13 @@ class LocalShards:
     def _step(self, inputs, expert_fn, stream):
         main = torch.cuda.current_stream()
 
-        def send(r, st):
+        def send(r, st):  # rows and counts into the owners' slabs
             rk, inp = self.ranks[r], inputs[r]
-            rk.layout(inp["topk_idx"], inp.get("x_active_mask"), st)
-            rk.dispatch(inp["x"], inp.get("smooth"), st)  # rows and counts into the owners' slabs
+            if self.fused:
+                rk.layout_dispatch(inp["topk_idx"], inp["x"], inp.get("x_active_mask"), inp.get("smooth"), st)
+            else:
+                rk.layout(inp["topk_idx"], inp.get("x_active_mask"), st)
+                rk.dispatch(inp["x"], inp.get("smooth"), st)
 
         def receive(r, st):
             rk, inp = self.ranks[r], inputs[r]
@@ -301,8 +314,7 @@ class DistShard:
 
     def _step(self, inp, expert_fn, stream):
         rk = self.rank
-        rk.layout(inp["topk_idx"], inp.get("x_active_mask"), stream)
-        rk.dispatch(inp["x"], inp.get("smooth"), stream)  # rows and counts into the owners' slabs
+        rk.layout_dispatch(inp["topk_idx"], inp["x"], inp.get("x_active_mask"), inp.get("smooth"), stream)
         self.group.barrier(self.device)  # every rank's dispatch is complete before the experts read
         if expert_fn is not None:
             expert_fn(self.slab, self.group.rank)

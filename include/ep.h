@@ -360,6 +360,17 @@ EP_API int ep_shard_dispatch(const ep_config* cfg, const ep_shard_table* tab, co
                              const float* smooth_scale, const int32_t* dst_pos, const int32_t* send_count,
                              float* token_scale, void* workspace, ep_stream_t stream);
 
+/* ep_shard_layout and ep_shard_dispatch of rank tab->rank as one call, with the count
+ * exchange (send_count stored into every owner's tab->recv_count column): same
+ * outputs.  When T <= 128 and k <= 8 all of it runs in one grid, as ep_layout_dispatch
+ * on one GPU: the first CTAs lay out the rank's tokens and store its counts, every
+ * other CTA derives one token's global rows from the routing and stores its copies;
+ * otherwise the two kernels run in order.  Arguments as for those two calls. */
+EP_API int ep_shard_layout_dispatch(const ep_config* cfg, const ep_shard_table* tab, const int32_t* topk_idx,
+                                    const uint8_t* x_active_mask, const uint16_t* x,
+                                    const float* smooth_scale, int32_t* dst_pos, int32_t* send_count,
+                                    float* token_scale, void* workspace, ep_stream_t stream);
+
 /* Combine of rank tab->rank's tokens into y (bf16 [T][d]); tab->recv_x[q] are the bf16
  * expert-output slabs; other arguments as ep_combine, local to this rank. */
 EP_API int ep_shard_combine(const ep_config* cfg, const ep_shard_table* tab,

@@ -219,6 +219,16 @@ def test_shard_calls_reject_bad_arguments_before_cuda():
     with pytest.raises(abi.EPError) as ei:
         abi.ep_shard_dispatch(c, good, fake, None, fake, fake + 2, fake, fake)
     assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    # layout and dispatch as one call: send_count and the workspace are required
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_layout_dispatch(c, good, fake, None, fake, None, fake, None, fake, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_layout_dispatch(c, good, fake, None, fake, None, fake, fake, fake, None)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
+    with pytest.raises(abi.EPError) as ei:
+        abi.ep_shard_layout_dispatch(c, holes, fake, None, fake, None, fake, fake, fake, fake)
+    assert ei.value.status == abi.EP_ERR_INVALID_ARG
     # combine: y must be given and must not be ori_x
     with pytest.raises(abi.EPError) as ei:
         abi.ep_shard_combine(c, good, fake, fake, None, fake, None, None, None, None, None, fake)

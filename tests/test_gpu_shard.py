@@ -124,12 +124,15 @@ def _check(w, sh, inp, ref, vals, compact, ys):
     rep.assert_ok()
 
 
+@pytest.mark.parametrize("fused", [True, False], ids=["one_call", "separate_calls"])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_shard_step_matches_oracle(dev, name):
+def test_shard_step_matches_oracle(dev, name, fused):
+    """Layout and dispatch as ep_shard_layout_dispatch (one grid for T <= 128, with the
+    count exchange in the layout CTAs) or as ep_shard_layout + ep_shard_dispatch."""
     w = CASES[name]
     if gp.need_bytes(w, True) > gp.free_bytes() - (4 << 30):
         pytest.skip("needs %.1f GB" % (gp.need_bytes(w, True) / 1e9))
-    _check(w, *_run(w, dev))
+    _check(w, *_run(w, dev, shards=shard.LocalShards(w, dev, fused=fused)))
 
 
 def test_shard_rank_streams(dev):
