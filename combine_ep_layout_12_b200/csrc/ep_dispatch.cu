@@ -609,13 +609,17 @@ int launch_dispatch(const Shape& s, const ep_buffer_ptrs& p, const uint16_t* x,
                     cudaStream_t stream) {
     if (s.B == 0) return EP_OK;
     DispatchArgs a = make_dispatch_args(s, p, x, smooth, topk_idx, active);
-    // Small batches per rank: each CTA derives its rows from the routing itself
-    // (at most kSelfRowsMaxT earlier tokens to scan), so dispatch overlaps layout.
-    // Packed rows also need the layout kernel's counts: ep_layout ends with the pack
-    // kernel, which starts only after the counting kernel has finished, so a
-    // dispatch started by the pack kernel can read them and run alongside it.
-    a.self_rows = (topk_idx != nullptr && s.T <= kSelfRowsMaxT) ? 1 : 0;
-    if (a.self_rows && s.layout == 1) {
+    // Where the rows come from.  Low-latency layout: dst_pos, read after the wait
+    // (one round trip; a CTA deriving its rows from the routing before the wait
+    // gains only while the layout kernel is still running, and a caller that wants
+    // that overlap has ep_layout_dispatch, whose one grid does it).  Packed layout,
+    // small batches per rank (at most kSelfRowsMaxT earlier tokens to scan): each
+    // CTA derives its rows from the routing and the first layout kernel's counts.
+    // ep_layout ends with the pack kernel, which starts only after the counting
+    // kernel has finished, so a dispatch started by the pack kernel can read them
+    // and run alongside it.
+    a.self_rows = (topk_idx != nullptr && s.layout == 1 && s.T <= kSelfRowsMaxT) ? 1 : 0;
+    if (a.self_rows) {
         a.expert_offset = p.expert_offset;
         a.recv_count = p.recv_count;
     }

@@ -208,17 +208,19 @@ EP_API int ep_layout(ep_buffer* buf, const int32_t* topk_idx, const uint8_t* x_a
  * (recv_count, expert_offset and recv_src), so one must have run on this buffer
  * (else EP_ERR_INVALID_ARG); it starts after the layout kernel has finished.  A
  * receive row whose recv_src is not a token sets EP_ERRBIT_ROW_RANGE and is skipped.
- * For T = B/P <= 256 the kernel derives those rows from the topk_idx (and mask)
- * passed to that ep_layout (which must still hold the same values) instead of reading dst_pos,
- * so it can run alongside the layout kernel (for the packed layout, alongside its
- * second kernel, reading the per-expert counts the first one wrote); it finishes
- * only after the layout kernels have.  Call it on the stream of that ep_layout, after it.
- * Ordering: in that small-batch form the kernel reads x and the routing and writes
- * recv_x, recv_scale and token_scale before it waits for the kernel ahead of it on
- * the stream.  That is safe because ep_layout's kernel waits for everything before
- * it first.  So no kernel that is launched with programmatic dependent launch and
- * triggers its dependents early may sit between ep_layout and ep_dispatch on the
- * stream (ordinary launches, copies and event waits may). */
+ * In the packed layout with T = B/P <= 256 the kernel derives those rows from the
+ * topk_idx (and mask) passed to that ep_layout (which must still hold the same
+ * values) and the per-expert counts its first kernel wrote, instead of reading
+ * dst_pos, so it can run alongside the layout's second kernel; it finishes only
+ * after the layout kernels have.  Call it on the stream of that ep_layout, after it.
+ * Ordering: in that packed small-batch form the kernel reads x, the routing and
+ * those counts and writes recv_x, recv_scale and token_scale before it waits for the
+ * kernel ahead of it on the stream.  That is safe because ep_layout's kernels wait
+ * for everything before them first.  So no kernel that is launched with
+ * programmatic dependent launch and triggers its dependents early may sit between
+ * ep_layout and ep_dispatch on the stream (ordinary launches, copies and event
+ * waits may).  In every other form the kernel waits before reading anything.
+ * (ep_layout_dispatch overlaps layout and dispatch in the low-latency layout.) */
 EP_API int ep_dispatch(ep_buffer* buf, const uint16_t* x, const float* smooth_scale,
                 ep_stream_t stream);
 
