@@ -240,11 +240,17 @@ EP_API int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx,
  * x_active_mask uint8 [B] or NULL, the mask given to ep_layout (inactive tokens
  * get y = +0);
  * ori_x bf16 [B][d] (required when C + K > 0, else may be NULL);
- * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos
- * (topk_idx must hold the ids given to that layout).
+ * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos,
+ * or for T = B/P <= 128 derives the same rows from topk_idx (which must hold the
+ * ids given to that layout) and the layout's counts.
  * y must not overlap any input.
- * Ordering: the kernel reads nothing before it waits for the kernel ahead of it on
- * the stream. */
+ * Ordering: in that small-batch form the kernel reads topk_idx, topk_weights,
+ * x_active_mask and (packed layout) expert_offset and recv_count before it waits for
+ * the kernel ahead of it on the stream, and reads expert outputs and writes y only
+ * after.  The library's own kernels before it (ep_layout, ep_dispatch) let it start
+ * only once those counts are final.  A kernel launched with programmatic dependent
+ * launch that triggers its dependents early and writes those inputs or counts must
+ * not be the one right before ep_combine on the stream. */
 EP_API int ep_combine(ep_buffer* buf, const uint16_t* expert_out, const int32_t* topk_idx,
                const float* topk_weights, const uint8_t* x_active_mask, const uint16_t* ori_x,
                const uint16_t* a1, const uint16_t* a2, const uint16_t* v, uint16_t* y,
