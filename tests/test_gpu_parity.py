@@ -526,6 +526,49 @@ def test_mask_rank0_decode(dev):
     assert rc[0].sum() == 0
 
 
+@pytest.mark.parametrize("T", [74, 75, 127])
+@pytest.mark.parametrize("qm", [1, 2])
+def test_dispatch_ragged_batches(dev, T, qm):
+    """Decode shape with per-rank batches that are not a power of two (592, 600 and
+    1016 tokens over 8 ranks), static and dynamic int8."""
+    w = wl.get("decode").with_(name="decode_T%d_q%d" % (T, qm), B=8 * T, M=T, quant_mode=qm,
+                               smooth="rand" if qm == 1 else "none")
+    full_check(w, dev)
+
+
+def test_dispatch_rewrites_every_row_on_every_call(dev):
+    """With the receive rows and scales overwritten by sentinels before every call,
+    each call of ep_dispatch writes every routed row and scale again, bit for bit as
+    the first, and the last one matches the oracle."""
+    w = wl.get("decode")
+    inp = wl.generate(w)
+    dev_inp = runner.to_device(inp, dev)
+    pipe = runner.Pipeline(w, dev)
+    pipe.layout(dev_inp)
+    torch.cuda.synchronize()
+    dp = pipe.buf.dst_pos.cpu().numpy()
+    rows = torch.from_numpy(dp[dp >= 0].astype(np.int64)).to(dev)
+    outs = []
+    for _ in range(4):
+        pipe.buf.recv_x.view(torch.uint8).fill_(0x5A)
+        pipe.buf.recv_scale.fill_(float("nan"))
+        pipe.buf.token_scale.fill_(float("nan"))
+        pipe.dispatch(dev_inp)
+        torch.cuda.synchronize()
+        outs.append((pipe.buf.recv_x[rows].clone(), pipe.buf.recv_scale[rows].clone(),
+                     pipe.buf.token_scale.clone()))
+    assert not torch.isnan(outs[0][1]).any() and not torch.isnan(outs[0][2]).any()
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
+    assert pipe.buf.check() == 0
+    # the last call against the oracle
+    rep = gp.Report()
+    ref = oracle.layout(gp.ocfg(w), inp["topk_idx"], active=inp.get("active"))
+    gp.check_dispatch(rep, w, pipe, inp, ref)
+    rep.assert_ok()
+
+
 def test_repeated_calls_are_identical(dev):
     """The layout's ticket counter re-arms itself; a second pass over the same
     inputs reproduces every output bit for bit and raises no error bits."""
