@@ -48,6 +48,8 @@ KERNEL_SOURCES = {  # every source file a kernel's code comes from
     "layout": [_CSRC + f for f in ("ep_layout.cu", "ep_layout_dev.cuh", "ep_internal.cuh")],
     "dispatch": [_CSRC + f for f in ("ep_dispatch.cu", "ep_dispatch_dev.cuh", "ep_internal.cuh")],
     "combine": [_CSRC + f for f in ("ep_combine.cu", "ep_internal.cuh")],
+    "layout_dispatch": [_CSRC + f for f in ("ep_fused.cu", "ep_layout_dev.cuh", "ep_dispatch_dev.cuh",
+                                            "ep_internal.cuh")],
 }
 
 
@@ -235,19 +237,22 @@ def source_hash(name, read=None):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, kernel):
+def recorded_traffic(workload, kernel, with_shape=False):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    the current kernel source (else None); with_shape: also the workload the
+    capture ran on (a smaller variant with the same per-launch traffic, or the
+    workload itself)."""
     path = os.path.join(PROFILES, "traffic.json")
     try:
         with open(path) as f:
             j = json.load(f)
         rec = j[workload][kernel]
         if rec.get("source_sha") != source_hash(kernel):
-            return None
-        return float(rec["dram_bytes_per_launch"])
+            return (None, None) if with_shape else None
+        b = float(rec["dram_bytes_per_launch"])
+        return (b, rec.get("captured_on", workload)) if with_shape else b
     except Exception:
-        return None
+        return (None, None) if with_shape else None
 
 
 def oracle_sample_prepare(w, inp, t0, n_tokens):
@@ -723,8 +728,10 @@ def run_ours(args):
                          "frac_of_measured": ach / peak, "frac_of_8tbs": ach / SPEC_HBM_GBS,
                          "share": ms / tot, "us_overlapped": 1e3 * kern_ms[name],
                          "achieved_gbs_overlapped": wb.kbytes[name] / (kern_ms[name] * 1e-3) / 1e9}
+    for name in kernels:
+        kernels[name]["traffic"], kernels[name]["traffic_captured_on"] = recorded_traffic(w.name, name, True)
     dom = max(("dispatch", "combine", "layout"), key=lambda n: kernels[n]["share"])
-    traffic = recorded_traffic(w.name, dom)
+    traffic = kernels[dom]["traffic"]
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["achieved_gbs"], "peak": peak,
                 "unit": "GB/s", "frac": kernels[dom]["achieved_gbs"] / peak, "traffic": traffic,
                 "peak_source": ("%s copy bandwidth (MEASURED_PEAKS.json hbm_gbs)" % peak_kind)
@@ -735,9 +742,13 @@ def run_ours(args):
                             "three times the L2 size, of the span between CUDA events around the launch, "
                             "minus the span of an empty event pair (%.2f us); raw span %.2f us"
                             % (1e3 * iso_ms["event_pair"], 1e3 * iso_ms["raw"][dom]),
+                "traffic_captured_on": kernels[dom]["traffic_captured_on"],
                 "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum of one ncu capture of this "
                                 "kernel (per launch), recorded in profiles/traffic.json; null once the "
-                                "kernel source has changed since"}
+                                "kernel source has changed since. traffic_captured_on names the workload "
+                                "the capture ran on: decode_e64 has the decode launch's tokens, hidden "
+                                "size, picks and routed rows (so its traffic per launch) on a 64-expert "
+                                "receive buffer that keeps the multi-pass capture near 1.4 GB"}
 
     # end to end through the public API with host buffers (eager calls, no graph).
     # Every step uploads its inputs from pinned host memory and reads its y back.
@@ -849,6 +860,7 @@ def run_ours(args):
         "layout_then_dispatch_us": 1e3 * kern_ms["layout+dispatch"],
         "layout_dispatch_one_call_us": 1e3 * kern_ms["layout_dispatch"],
         "layout_dispatch_one_call_us_isolated": 1e3 * iso_ms["layout_dispatch"],
+        "layout_dispatch_one_call_traffic": recorded_traffic(w.name, "layout_dispatch"),
         "comm_gbs_dispatch": wb.n_routed * w.d * (1 if w.quant_mode != 0 else 2)
         / (kern_ms["dispatch"] * 1e-3) / 1e9,
         "roofline": roofline,

@@ -2,6 +2,7 @@
 recorded-traffic lookup and its staleness rule, and the seeded inputs the
 measurements are taken on."""
 import json
+import os
 
 import numpy as np
 
@@ -25,6 +26,26 @@ def test_recorded_traffic_follows_the_source(tmp_path, monkeypatch):
     assert bench.recorded_traffic("w", "combine") == 123.0
     assert bench.recorded_traffic("w", "dispatch") is None      # taken on other kernel source
     assert bench.recorded_traffic("other", "combine") is None
+    assert bench.recorded_traffic("w", "combine", with_shape=True) == (123.0, "w")
+    assert bench.recorded_traffic("w", "dispatch", with_shape=True) == (None, None)
+
+
+def test_committed_traffic_records_name_known_kernels():
+    """Every record of the committed traffic file belongs to a kernel whose sources
+    the benchmark hashes, with the bytes, the hash and the workload it was taken on."""
+    with open(os.path.join(bench.PROFILES, "traffic.json")) as f:
+        doc = json.load(f)
+    n = 0
+    for wname, recs in doc.items():
+        if wname.startswith("_"):
+            continue
+        for kern, rec in recs.items():
+            assert kern in bench.KERNEL_SOURCES, (wname, kern)
+            assert rec["dram_bytes_per_launch"] > 0
+            assert len(rec["source_sha"]) == 16 and rec["captured_on"]
+            n += 1
+    assert "layout_dispatch" in doc["decode"]
+    assert n >= 10
 
 
 def test_source_hash_ignores_comments_only():
