@@ -22,10 +22,17 @@
 namespace ep {
 namespace {
 
-// Per-rank batches up to this size derive their rows from the routing (the scan of
-// the earlier tokens' ids stays within one load per thread).  At 256 tokens per
-// rank reading dst_pos was measured faster (90 against 102 us per combine at
-// P = 16, d = 7168, k = 8): the scan's L2 reads grow with T while dst_pos does not.
+// Where the receive rows come from.  The routing scan runs before
+// griddepcontrol.wait, so it is hidden only while a preceding kernel of the
+// library still runs; otherwise its cost is exposed (about 1 us at decode, more
+// than the one round trip of reading dst_pos after the wait).  In a model the
+// combine follows the expert kernels, so dst_pos is the default.  The scan is kept
+// where it measured faster in back-to-back steps: per-rank batches of at most
+// kCombineScanMaxT tokens (few earlier tokens to scan), and, up to
+// kCombineSelfRowsMaxT tokens, buffers with a per-expert smooth table, whose
+// persistent dispatch kernel drains while the scan runs (56.5 against 63.0 us per
+// step at decode).  Above kCombineSelfRowsMaxT the scan's L2 reads grow with T.
+constexpr int kCombineScanMaxT = 16;
 constexpr int kCombineSelfRowsMaxT = 128;
 
 struct CombineArgs {
@@ -223,7 +230,8 @@ int launch_combine_impl(const Shape& s, const ep_buffer_ptrs& p, const uint16_t*
     a.M = s.M;
     // packed rows also read the layout's counts, complete before the dispatch that
     // precedes this kernel started
-    a.self_rows = (tab == nullptr && s.T <= kCombineSelfRowsMaxT) ? 1 : 0;
+    a.self_rows = (tab == nullptr && (s.T <= kCombineScanMaxT ||
+                                      (s.expert_smooth && s.T <= kCombineSelfRowsMaxT))) ? 1 : 0;
     a.expert_offset = (a.self_rows && s.layout == 1) ? p.expert_offset : nullptr;
     a.recv_count = (a.self_rows && s.layout == 1) ? p.recv_count : nullptr;
     // One CTA per token when that fills the GPU in about one wave; otherwise split

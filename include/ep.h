@@ -241,8 +241,9 @@ EP_API int ep_layout_dispatch(ep_buffer* buf, const int32_t* topk_idx,
  * get y = +0);
  * ori_x bf16 [B][d] (required when C + K > 0, else may be NULL);
  * a1, a2, v bf16 [K][d] (required iff K > 0).  Uses the latest layout's dst_pos,
- * or for T = B/P <= 128 derives the same rows from topk_idx (which must hold the
- * ids given to that layout) and the layout's counts.
+ * or, for T = B/P <= 16 and for T <= 128 on a buffer with a per-expert smooth table
+ * (smooth_rows > 1), derives the same rows from topk_idx (which must hold the ids
+ * given to that layout) and the layout's counts.
  * y must not overlap any input.
  * Ordering: in that small-batch form the kernel reads topk_idx, topk_weights,
  * x_active_mask and (packed layout) expert_offset and recv_count before it waits for
